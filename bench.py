@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Benchmark of the routed MoE FFN layer (DeepSeek-V4-Flash, MXFP4 experts,
+int8 shared expert) on B200: prints ONE JSON line.
+
+A step is one pass of the whole layer -- route, permute, forward -- over one
+synthetic batch of the chosen workload (default: the full-size layer at decode
+batch 1). Inputs are resident in HBM when timing starts; L2 is flushed
+(512 MiB write) between timed steps; every step is timed with CUDA events on
+the launch stream and the sum over steps is taken, max over ranks.
+
+Multi-GPU: replicas only (one process per GPU, each runs its own batch; no
+collective on the data path), launched with torch.distributed.run.
+
+`--impl reference` times the CPU oracle (the plain fp64 definition) on a
+bounded sample of the same workload and prints the same line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_b1")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def expert_bytes(wl):
+    w13 = 2 * wl.I * wl.H // 2 + 2 * wl.I * wl.H // 32
+    w2 = wl.H * wl.I // 2 + wl.H * wl.I // 32
+    return w13, w2
+
+
+def shared_bytes(wl):
+    if wl.Is == 0:
+        return 0, 0
+    return 2 * wl.Is * wl.H + 2 * wl.Is * 4, wl.H * wl.Is + wl.H * 4
+
+
+def algorithmic(wl, ids, token_ids=None):
+    """Algorithmic bytes/FLOPs of one step and of each kernel kind."""
+    T, H, I, Is, E, k = wl.T, wl.H, wl.I, wl.Is, wl.E, wl.k
+    S = T * k
+    n_hit = int(len(np.unique(ids))) if ids.size else 0
+    e13, e2 = expert_bytes(wl)
+    s13, s2 = shared_bytes(wl)
+    route_b = E * H * 2 + E * 4                     # gate + bias
+    if wl.routing == "hash":
+        n_tok = int(len(np.unique(token_ids))) if token_ids is not None else T
+        route_b = E * H * 2 + T * 4 + n_tok * k * 4  # gate + token ids + touched table rows
+    step_b = n_hit * (e13 + e2) + s13 + s2 + route_b + 4 * T * H + 48 * T
+    flops = S * 6 * H * I + T * 6 * H * Is + 2 * T * E * H
+    per_kernel_bytes = {
+        "w13": n_hit * e13 + s13 + T * H * 2 + S * I * 2 + T * Is * 2,
+        "w2": n_hit * e2 + s2 + S * I * 2 + T * Is * 2 + T * H * 2,
+    }
+    per_kernel_flops = {
+        "w13": S * 2 * (2 * I) * H + T * 2 * (2 * Is) * H,
+        "w2": S * 2 * H * I + T * 2 * H * Is,
+    }
+    return dict(n_hit=n_hit, step_bytes=step_b, step_flops=flops, kernel_bytes=per_kernel_bytes,
+                kernel_flops=per_kernel_flops)
+
+
+def kernel_kind(name):
+    if "w13" in name:
+        return "w13"
+    if "w2" in name:
+        return "w2"
+    return None
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def csrc_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "mxfp4_routed_expert_v4moe_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(f"{kernel}@{workload}")
+        if e and e.get("csrc") == csrc_hash():
+            return e.get("bytes_per_launch")
+    except Exception:
+        return None
+    return None
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.uuid and self.uuid not in parts[0]:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(wl, li, n_tok, seconds):
+    """Time the oracle (route + layer) on n_tok tokens of the workload, repeated
+    until about `seconds` of CPU time; returns (tokens/s, tokens, reps, secs)."""
+    import inputs as IN
+    import oracle as O
+    toks = np.arange(min(n_tok, wl.T), dtype=np.int32)
+    sub = IN.LayerInputs(wl=wl.with_T(len(toks)), x=np.ascontiguousarray(li.x[toks]), gate=li.gate,
+                         bias=li.bias,
+                         token_ids=None if li.token_ids is None else np.ascontiguousarray(li.token_ids[toks]),
+                         tid2eid=li.tid2eid, w13_codes=li.w13_codes, w13_scales=li.w13_scales,
+                         w2_codes=li.w2_codes, w2_scales=li.w2_scales, sh13=li.sh13,
+                         sh13_scale=li.sh13_scale, sh2=li.sh2, sh2_scale=li.sh2_scale)
+    lay = O.Layer(sub)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        ids, w, _, _ = lay.route()
+        lay.moe_tokens(np.arange(len(toks)), ids, w, threads=1)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return reps * len(toks) / el, len(toks), reps, el
+
+
+# ----------------------------------------------------------------------------- main
+
+def run_reference(args):
+    import inputs as IN
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = IN.WORKLOADS[args.workload]
+    li = IN.make_layer_inputs(wl)
+    step_times = []
+    n_tok = 1
+    for i in range(args.warmup + args.steps):
+        tps, ntk, reps, el = oracle_sample(wl, li, n_tok, 0.0)
+        if i >= args.warmup:
+            step_times.append(el / reps)
+    ms = 1e3 * float(np.mean(step_times))
+    value = n_tok / (ms / 1e3)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                       "shared_inter": wl.Is, "routing": wl.routing},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{n_tok} token(s) of {wl.name} per step (route over all "
+                                       f"{wl.E} experts + {wl.k} routed experts + shared expert)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+
+    import inputs as IN
+    import mxfp4_routed_expert_v4moe_b200 as V
+    from mxfp4_routed_expert_v4moe_b200 import MoELayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    wl = IN.WORKLOADS[args.workload]
+    li = IN.make_layer_inputs(wl)
+    layer = MoELayer.from_host(li, device=dev)
+    x = torch.from_numpy(li.x).view(torch.bfloat16).to(dev)
+    bias = None if li.bias is None else torch.from_numpy(li.bias).to(dev)
+    tok = None if li.token_ids is None else torch.from_numpy(li.token_ids).to(dev)
+    tab = None if li.tid2eid is None else torch.from_numpy(li.tid2eid).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        return layer(x, bias, tok, tab)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ids_np = layer.buffers(wl.T)["topk_ids"].cpu().numpy()
+    acc = algorithmic(wl, ids_np, li.token_ids)
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+
+    # ---- timed region: K steps, L2 flushed between steps ----------------------
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = V.v4moe_launch_count()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    launches = V.v4moe_launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    ms_total = sum(a.elapsed_time(b) for a, b in evs)
+
+    # ---- end to end through the public API: pinned host in, host out ----------
+    x_host = torch.from_numpy(li.x).view(torch.bfloat16).pin_memory()
+    tok_host = None if li.token_ids is None else torch.from_numpy(li.token_ids).pin_memory()
+    out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    tok_dev = None if tok is None else torch.empty_like(tok)
+    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e2e_evs[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        if tok_dev is not None:
+            tok_dev.copy_(tok_host, non_blocking=True)
+        out = layer(x_dev, bias, tok_dev, tab)
+        out_host.copy_(out, non_blocking=True)
+        e2e_evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs)
+    clk = clocks.stop()
+
+    # ---- per-kernel timing pass (events around every kernel) -----------------
+    V.v4moe_profile_reset()
+    V.v4moe_profile_enable(True)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize(dev)
+    prof = V.v4moe_profile_read()
+    V.v4moe_profile_enable(False)
+
+    t_ms = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_ms, op=dist.ReduceOp.MAX)
+    ms_total, e2e_ms = float(t_ms[0]), float(t_ms[1])
+    ms_step = ms_total / args.steps
+    tokens_total = wl.T * world
+    value = tokens_total / (ms_step / 1e3)
+    e2e_value = tokens_total / (e2e_ms / args.steps / 1e3)
+
+    pk = peaks()
+    decode = wl.T <= 64
+    # dominant kernel = most device time in the profiled pass
+    dom_name, (dom_ms, dom_n) = max(prof.items(), key=lambda kv: kv[1][0]) if prof else ("none", (0.0, 1))
+    kind = kernel_kind(dom_name)
+    per_launch_s = dom_ms / max(dom_n, 1) / 1e3
+    steps_per_launch = max(dom_n, 1) / args.steps
+    if decode or kind is None:
+        alg = acc["kernel_bytes"].get(kind, acc["step_bytes"]) / steps_per_launch
+        achieved = alg / per_launch_s / 1e9 if per_launch_s > 0 else 0.0
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "peak_src": pk["src"]}
+    else:
+        alg = acc["kernel_flops"][kind] / steps_per_launch
+        achieved = alg / per_launch_s / 1e12 if per_launch_s > 0 else 0.0
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16"], "peak_src": pk["src"]}
+    roof.update(kernel=dom_name, kernel_ms=dom_ms / max(dom_n, 1), algorithmic_per_launch=alg,
+                traffic=recorded_traffic(dom_name, wl.name))
+    step_s = ms_step / 1e3
+    layer_roof_s = max(acc["step_bytes"] / (pk["hbm"] * 1e9), acc["step_flops"] / (pk["bf16"] * 1e12))
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+                       "shared_inter": wl.Is, "routing": wl.routing, "global_batch": wl.T * world,
+                       "parallelism": f"replicas{world}", "experts_hit": acc["n_hit"],
+                       "l2": "flushed between timed steps (512 MiB write)",
+                       "weights": "MXFP4 routed (E2M1 + E8M0/32), int8 shared, bf16 gate"},
+            "layer_roofline": {"algorithmic_bytes": acc["step_bytes"],
+                               "algorithmic_flops": acc["step_flops"],
+                               "roofline_ms": layer_roof_s * 1e3,
+                               "frac": layer_roof_s / step_s,
+                               "achieved_GBps": acc["step_bytes"] / step_s / 1e9,
+                               "achieved_TFLOPs": acc["step_flops"] / step_s / 1e12},
+            "roofline": roof,
+            "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches_per_step": v[1] / args.steps}
+                        for k, v in sorted(prof.items(), key=lambda kv: -kv[1][0])},
+            "e2e": {"value": e2e_value, "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(x_host.numel() * 2 + (0 if tok_host is None else tok_host.numel() * 4)),
+                    "d2h_bytes_per_step": int(out_host.numel() * 2)},
+            "gpu_launches": int(launches),
+            "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, ntk, reps, el = oracle_sample(wl, li, 1, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{reps} x {ntk} token(s) of {wl.name} (route over all "
+                                          f"{wl.E} experts + layer), {el:.1f} s single-threaded fp64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

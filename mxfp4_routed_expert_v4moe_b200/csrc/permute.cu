@@ -1,0 +1,183 @@
+// Token permutation by expert: a deterministic, stable counting sort of the
+// T*k (token, slot) pairs by expert id, which groups the rows each expert's
+// GEMM consumes (the experts(flat, indices, weights) step of the MoE block,
+// "Checked in its code" row "Shared expert").
+//
+// Small inputs (T*k <= kPermChunk): one CTA does histogram, scan and scatter.
+// Large inputs: per-chunk histograms (one CTA per chunk of kPermChunk slots),
+// one CTA scans experts and chunk bases, then one warp per chunk scatters its
+// slots in order. Stability inside a chunk comes from walking the chunk in
+// slot order, 32 slots at a time, with __match_any_sync ranking equal ids.
+#include "launch.cuh"
+#include "v4moe_internal.cuh"
+
+namespace v4moe {
+namespace {
+
+__device__ __forceinline__ bool id_ok(int e, int E) { return e >= 0 && e < E; }
+
+// Walks slots [s0, s1) in order with one warp; cursor[e] (shared) holds the
+// next output position of expert e and is advanced.
+__device__ __forceinline__ void warp_stable_scatter(const int32_t* __restrict__ ids, int s0, int s1,
+                                                    int E, int* cursor, int32_t* __restrict__ sorted_slot,
+                                                    int32_t* __restrict__ slot_pos) {
+  const int lane = threadIdx.x & 31;
+  for (int base = s0; base < s1; base += 32) {
+    const int s = base + lane;
+    int e = -1;
+    if (s < s1) {
+      e = ids[s];
+      if (!id_ok(e, E)) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int pos = 0;
+    if (e >= 0) pos = cursor[e] + rank;
+    __syncwarp();
+    if (e >= 0) {
+      const int leader = __ffs(peers) - 1;
+      if (lane == leader) cursor[e] += __popc(peers);
+      sorted_slot[pos] = s;
+      slot_pos[s] = pos;
+    }
+    __syncwarp();
+  }
+}
+
+// Exclusive scan of v over the block (blockDim.x == 1024, one value per
+// thread); returns the exclusive prefix, *total gets the sum.
+__device__ int block_exclusive_scan(int v, int* total) {
+  __shared__ int warp_sums[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    warp_sums[lane] = wi - w;  // exclusive over warps
+  }
+  __syncthreads();
+  const int excl = warp_sums[warp] + incl - v;
+  // total: last thread's inclusive value
+  __shared__ int tot;
+  if (threadIdx.x == blockDim.x - 1) tot = excl + v;
+  __syncthreads();
+  *total = tot;
+  return excl;
+}
+
+__global__ void __launch_bounds__(1024) k_perm_single(int S, int E, const int32_t* __restrict__ ids,
+                                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                     int32_t* __restrict__ sorted_slot,
+                                                     int32_t* __restrict__ slot_pos, uint32_t* status) {
+  __shared__ int cnt[1024];
+  __shared__ int cursor[1024];
+  cnt[threadIdx.x] = 0;
+  __syncthreads();
+  bool bad = false;
+  for (int s = threadIdx.x; s < S; s += blockDim.x) {
+    const int e = ids[s];
+    if (id_ok(e, E))
+      atomicAdd(&cnt[e], 1);
+    else
+      bad = true;
+  }
+  if (bad) atomicOr(status, kStatusBadExpertId);
+  __syncthreads();
+  const int v = threadIdx.x < E ? cnt[threadIdx.x] : 0;
+  int total;
+  const int excl = block_exclusive_scan(v, &total);
+  if (threadIdx.x < E) {
+    counts[threadIdx.x] = v;
+    offsets[threadIdx.x] = excl;
+    cursor[threadIdx.x] = excl;
+  }
+  if (threadIdx.x == 0) offsets[E] = total;
+  __syncthreads();
+  if (threadIdx.x < 32) warp_stable_scatter(ids, 0, S, E, cursor, sorted_slot, slot_pos);
+}
+
+__global__ void __launch_bounds__(256) k_perm_hist(int S, int E, const int32_t* __restrict__ ids,
+                                                   int32_t* __restrict__ chunk_counts, uint32_t* status) {
+  __shared__ int cnt[1024];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int s0 = blockIdx.x * kPermChunk, s1 = min(S, s0 + kPermChunk);
+  bool bad = false;
+  for (int s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
+    const int e = ids[s];
+    if (id_ok(e, E))
+      atomicAdd(&cnt[e], 1);
+    else
+      bad = true;
+  }
+  if (bad) atomicOr(status, kStatusBadExpertId);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[size_t(blockIdx.x) * E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(1024) k_perm_scan(int E, int nchunks, const int32_t* __restrict__ chunk_counts,
+                                                    int32_t* __restrict__ chunk_base,
+                                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  const int e = threadIdx.x;
+  int tot = 0;
+  if (e < E)
+    for (int c = 0; c < nchunks; ++c) tot += chunk_counts[size_t(c) * E + e];
+  int total;
+  const int excl = block_exclusive_scan(e < E ? tot : 0, &total);
+  if (e < E) {
+    counts[e] = tot;
+    offsets[e] = excl;
+    int run = excl;
+    for (int c = 0; c < nchunks; ++c) {
+      chunk_base[size_t(c) * E + e] = run;
+      run += chunk_counts[size_t(c) * E + e];
+    }
+  }
+  if (threadIdx.x == 0) offsets[E] = total;
+}
+
+__global__ void __launch_bounds__(32) k_perm_scatter(int S, int E, const int32_t* __restrict__ ids,
+                                                     const int32_t* __restrict__ chunk_base,
+                                                     int32_t* __restrict__ sorted_slot,
+                                                     int32_t* __restrict__ slot_pos) {
+  __shared__ int cursor[1024];
+  for (int e = threadIdx.x; e < E; e += 32) cursor[e] = chunk_base[size_t(blockIdx.x) * E + e];
+  __syncwarp();
+  const int s0 = blockIdx.x * kPermChunk, s1 = min(S, s0 + kPermChunk);
+  warp_stable_scatter(ids, s0, s1, E, cursor, sorted_slot, slot_pos);
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const v4moe_config& c, int T, const int32_t* topk_ids, int32_t* counts,
+                           int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos,
+                           int32_t* chunk_counts, int32_t* chunk_base, int nchunks,
+                           uint32_t* status, cudaStream_t st) {
+  const int S = T * c.top_k;
+  const int E = c.n_experts;
+  if (S <= kPermChunk)
+    return launch_kernel("perm_single", k_perm_single, dim3(1), dim3(1024), 0, st, false, S, E, topk_ids,
+                         counts, offsets, sorted_slot, slot_pos, status);
+  cudaError_t e = launch_kernel("perm_hist", k_perm_hist, dim3(nchunks), dim3(256), 0, st, false, S, E,
+                                topk_ids, chunk_counts, status);
+  if (e != cudaSuccess) return e;
+  e = launch_kernel("perm_scan", k_perm_scan, dim3(1), dim3(1024), 0, st, false, E, nchunks,
+                    (const int32_t*)chunk_counts, chunk_base, counts, offsets);
+  if (e != cudaSuccess) return e;
+  return launch_kernel("perm_scatter", k_perm_scatter, dim3(nchunks), dim3(32), 0, st, false, S, E, topk_ids,
+                       (const int32_t*)chunk_base, sorted_slot, slot_pos);
+}
+
+}  // namespace v4moe

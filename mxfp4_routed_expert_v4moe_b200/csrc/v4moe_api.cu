@@ -1,0 +1,191 @@
+// C-ABI entry points of libv4moe: argument validation, workspace carve-up and
+// dispatch to the kernels. The declarations and their contracts are in
+// include/v4moe.h.
+#include <mutex>
+#include <unordered_map>
+
+#include "v4moe_internal.cuh"
+
+namespace v4moe {
+
+cudaError_t launch_forward_simt(const ForwardArgs& a, cudaStream_t st);
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool config_ok(const v4moe_config* c) {
+  if (!c) return false;
+  if (c->hidden <= 0 || c->hidden % 128 != 0) return false;
+  if (c->inter <= 0 || c->inter % 128 != 0) return false;
+  if (c->shared_inter < 0 || c->shared_inter % 128 != 0) return false;
+  if (c->top_k < 1 || c->top_k > 8) return false;
+  if (c->n_experts < c->top_k || c->n_experts > 1024) return false;
+  if (!(c->routed_scale == c->routed_scale) || !(c->swiglu_limit > 0.0f)) return false;
+  return true;
+}
+
+// Per-device compute capability cache.
+int32_t check_device() {
+  static std::mutex mu;
+  static std::unordered_map<int, bool> ok;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return V4MOE_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = ok.find(dev);
+  if (it == ok.end()) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return V4MOE_ERR_UNSUPPORTED_DEVICE;
+    }
+    it = ok.emplace(dev, major == 10 && minor == 0).first;
+  }
+  return it->second ? V4MOE_OK : V4MOE_ERR_UNSUPPORTED_DEVICE;
+}
+
+int32_t check_ws(const v4moe_config* c, int32_t T, const void* ws, size_t ws_bytes) {
+  if (!ws || !aligned(ws, 256)) return V4MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(*c, T).total) return V4MOE_ERR_WORKSPACE;
+  return V4MOE_OK;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+int32_t launch_status(cudaError_t e) {
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return V4MOE_ERR_LAUNCH;
+  }
+  return V4MOE_OK;
+}
+
+}  // namespace
+}  // namespace v4moe
+
+using namespace v4moe;
+
+extern "C" {
+
+size_t v4moe_workspace_bytes(const v4moe_config* cfg, int32_t T) {
+  if (!config_ok(cfg) || T < 0) return 0;
+  return ws_layout(*cfg, T).total;
+}
+
+int32_t v4moe_route(const v4moe_config* cfg, int32_t T, const void* x, const void* gate,
+                    const float* bias, const int32_t* token_ids, const int32_t* tid2eid,
+                    int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  if (!config_ok(cfg) || T < 0) return V4MOE_ERR_INVALID_ARG;
+  const bool hash = token_ids != nullptr || tid2eid != nullptr;
+  if (hash && (bias || !token_ids || !tid2eid || cfg->vocab <= 0)) return V4MOE_ERR_INVALID_ARG;
+  if (!hash && !bias) return V4MOE_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!x || !gate || !topk_ids || !topk_w) return V4MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(gate, 16) || !aligned(topk_ids, 4) || !aligned(topk_w, 4))
+      return V4MOE_ERR_INVALID_ARG;
+  }
+  if (int32_t r = check_ws(cfg, T, ws, ws_bytes)) return r;
+  if (int32_t r = check_device()) return r;
+  if (T == 0) return V4MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  return launch_status(launch_route(*cfg, T, static_cast<const __nv_bfloat16*>(x),
+                                    static_cast<const __nv_bfloat16*>(gate), bias, token_ids, tid2eid,
+                                    topk_ids, topk_w, at<float>(ws, L.scores), at<uint32_t>(ws, L.status),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int32_t v4moe_permute(const v4moe_config* cfg, int32_t T, const int32_t* topk_ids, int32_t* counts,
+                      int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos, void* ws,
+                      size_t ws_bytes, void* stream) {
+  if (!config_ok(cfg) || T < 0) return V4MOE_ERR_INVALID_ARG;
+  if (!counts || !offsets) return V4MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_ids || !sorted_slot || !slot_pos)) return V4MOE_ERR_INVALID_ARG;
+  if (int64_t(T) * cfg->top_k > 0x7fffffff / 2) return V4MOE_ERR_INVALID_ARG;
+  if (int32_t r = check_ws(cfg, T, ws, ws_bytes)) return r;
+  if (int32_t r = check_device()) return r;
+  const WsLayout L = ws_layout(*cfg, T);
+  return launch_status(launch_permute(*cfg, T, topk_ids, counts, offsets, sorted_slot, slot_pos,
+                                      at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.chunk_base),
+                                      L.nchunks, at<uint32_t>(ws, L.status),
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x, const int32_t* topk_ids,
+                      const float* topk_w, const int32_t* offsets, const int32_t* sorted_slot,
+                      const int32_t* slot_pos, const v4moe_weights* weights, void* out, void* ws,
+                      size_t ws_bytes, void* stream) {
+  if (!config_ok(cfg) || T < 0 || !weights) return V4MOE_ERR_INVALID_ARG;
+  const v4moe_weights& w = *weights;
+  if (!w.w13_codes || !w.w13_scales || !w.w2_codes || !w.w2_scales) return V4MOE_ERR_INVALID_ARG;
+  if (!aligned(w.w13_codes, 16) || !aligned(w.w2_codes, 16) || !aligned(w.w13_scales, 4) ||
+      !aligned(w.w2_scales, 4))
+    return V4MOE_ERR_INVALID_ARG;
+  if (cfg->shared_inter > 0) {
+    if (!w.sh_w13 || !w.sh_w13_scale || !w.sh_w2 || !w.sh_w2_scale) return V4MOE_ERR_INVALID_ARG;
+    if (!aligned(w.sh_w13, 16) || !aligned(w.sh_w2, 16)) return V4MOE_ERR_INVALID_ARG;
+  }
+  if (!offsets) return V4MOE_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!x || !topk_ids || !topk_w || !sorted_slot || !slot_pos || !out) return V4MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16)) return V4MOE_ERR_INVALID_ARG;
+    if (x == out) return V4MOE_ERR_INVALID_ARG;
+  }
+  if (int32_t r = check_ws(cfg, T, ws, ws_bytes)) return r;
+  if (int32_t r = check_device()) return r;
+  if (T == 0) return V4MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  ForwardArgs a;
+  a.c = *cfg;
+  a.T = T;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.topk_ids = topk_ids;
+  a.topk_w = topk_w;
+  a.offsets = offsets;
+  a.sorted_slot = sorted_slot;
+  a.slot_pos = slot_pos;
+  a.w = w;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.status = at<uint32_t>(ws, L.status);
+  a.h = at<__nv_bfloat16>(ws, L.h);
+  a.y_slot = at<float>(ws, L.y_slot);
+  a.hs = at<__nv_bfloat16>(ws, L.hs);
+  a.ys = at<float>(ws, L.ys);
+  return launch_status(launch_forward_simt(a, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t v4moe_read_device_status(const void* ws, void* stream) {
+  if (!ws || !aligned(ws, 256)) return V4MOE_ERR_INVALID_ARG;
+  uint32_t word = 0;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess ||
+      cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return V4MOE_ERR_LAUNCH;
+  }
+  if (word & kStatusTimeout) return V4MOE_ERR_TIMEOUT;
+  if (word & (kStatusBadExpertId | kStatusBadTokenId)) return V4MOE_ERR_DATA;
+  return V4MOE_OK;
+}
+
+int32_t v4moe_clear_device_status(void* ws, void* stream) {
+  if (!ws || !aligned(ws, 256)) return V4MOE_ERR_INVALID_ARG;
+  return launch_status(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)));
+}
+
+const char* v4moe_status_string(int32_t s) {
+  switch (s) {
+    case V4MOE_OK: return "ok";
+    case V4MOE_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer or bad shape)";
+    case V4MOE_ERR_WORKSPACE: return "workspace too small";
+    case V4MOE_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs compute capability 10.0)";
+    case V4MOE_ERR_LAUNCH: return "kernel launch failed";
+    case V4MOE_ERR_DATA: return "device flagged out-of-range expert or token ids";
+    case V4MOE_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

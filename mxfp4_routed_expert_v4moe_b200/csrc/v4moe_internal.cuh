@@ -1,0 +1,113 @@
+// Internal declarations shared by the libv4moe translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/v4moe.h"
+
+namespace v4moe {
+
+// Device status word bits (first 4 bytes of the workspace).
+constexpr uint32_t kStatusBadExpertId = 1u << 0;
+constexpr uint32_t kStatusBadTokenId = 1u << 1;
+constexpr uint32_t kStatusTimeout = 1u << 2;
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a; }
+
+// Slots per chunk of the multi-CTA permutation.
+constexpr int kPermChunk = 2048;
+
+// Workspace carve-up for T tokens. All offsets are 256-byte aligned.
+struct WsLayout {
+  size_t status = 0;        // uint32 status word + spare words (256 B)
+  size_t scores = 0;        // [T, E] fp32 router scores
+  size_t chunk_counts = 0;  // [nchunks, E] int32
+  size_t chunk_base = 0;    // [nchunks, E] int32
+  size_t h = 0;             // [T*k, I] bf16 routed intermediates (sorted order)
+  size_t y_slot = 0;        // [T*k, H] fp32 routed expert outputs (sorted order)
+  size_t hs = 0;            // [T, I_s] bf16 shared intermediates
+  size_t ys = 0;            // [T, H] fp32 shared expert outputs
+  size_t total = 0;
+  int nchunks = 0;
+};
+
+inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
+  WsLayout L;
+  const int64_t S = T * c.top_k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  L.status = take(256);
+  L.scores = take(size_t(T) * c.n_experts * 4);
+  L.nchunks = int((S + kPermChunk - 1) / kPermChunk);
+  if (L.nchunks < 1) L.nchunks = 1;
+  L.chunk_counts = take(size_t(L.nchunks) * c.n_experts * 4);
+  L.chunk_base = take(size_t(L.nchunks) * c.n_experts * 4);
+  L.h = take(size_t(S) * c.inter * 2);
+  L.y_slot = take(size_t(S) * c.hidden * 4);
+  L.hs = take(size_t(T) * (c.shared_inter > 0 ? c.shared_inter : 0) * 2);
+  L.ys = take(size_t(T) * c.hidden * 4);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- launchers
+// Each returns cudaGetLastError() of its launches.
+cudaError_t launch_route(const v4moe_config& c, int T, const __nv_bfloat16* x,
+                         const __nv_bfloat16* gate, const float* bias, const int32_t* token_ids,
+                         const int32_t* tid2eid, int32_t* topk_ids, float* topk_w, float* scores,
+                         uint32_t* status, cudaStream_t st);
+
+cudaError_t launch_permute(const v4moe_config& c, int T, const int32_t* topk_ids, int32_t* counts,
+                           int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos,
+                           int32_t* chunk_counts, int32_t* chunk_base, int nchunks,
+                           uint32_t* status, cudaStream_t st);
+
+struct ForwardArgs {
+  v4moe_config c;
+  int T;
+  const __nv_bfloat16* x;
+  const int32_t* topk_ids;
+  const float* topk_w;
+  const int32_t* offsets;
+  const int32_t* sorted_slot;
+  const int32_t* slot_pos;
+  v4moe_weights w;
+  __nv_bfloat16* out;
+  // workspace pieces
+  uint32_t* status;
+  __nv_bfloat16* h;
+  float* y_slot;
+  __nv_bfloat16* hs;
+  float* ys;
+};
+
+cudaError_t launch_forward_simt(const ForwardArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- device helpers
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// sqrt(softplus(z)) in fp32, softplus in its overflow-free form.
+__device__ __forceinline__ float sqrt_softplus_f(float z) {
+  const float sp = fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
+  return sqrtf(sp);
+}
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.0f + expf(-v)); }
+
+// Clamped SwiGLU: gate clamped from above, up on both sides.
+__device__ __forceinline__ float clamped_swiglu_f(float g, float u, float limit) {
+  const float gc = fminf(g, limit);
+  const float uc = fminf(fmaxf(u, -limit), limit);
+  return silu_f(gc) * uc;
+}
+
+}  // namespace v4moe

@@ -176,7 +176,7 @@ class Layer:
         if threads == 1:
             run(0, n)
         else:
-            bounds = np.linspace(0, n, threads + 1).astype(int)
+            bounds = [int(b) for b in np.linspace(0, n, threads + 1).round()]
             with ThreadPoolExecutor(threads) as ex:
                 list(ex.map(lambda i: run(bounds[i], bounds[i + 1]), range(threads)))
         if want_h:

@@ -1,0 +1,164 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs. Integer outputs bit-exact (learned-routing tokens whose
+6th-vs-7th biased-score margin is below 1e-4 are counted and left out of the id
+comparison); float outputs within rel-L2 5e-3 and max-abs 1e-2 * max|ref|."""
+import numpy as np
+import pytest
+
+import inputs as IN
+import oracle as O
+from parity_util import (NEAR_TIE, assert_close, bf16_to_f64, host_threads, sample_tokens,
+                         upload_activations)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _layer(li):
+    from mxfp4_routed_expert_v4moe_b200 import MoELayer
+    return MoELayer.from_host(li)
+
+
+@pytest.fixture(scope="module")
+def full_weights():
+    """Full-size weights (identical for every full-size workload, seed 0)."""
+    return IN.make_weights(IN.WORKLOADS["decode_b1"])
+
+
+def run_parity(li, layer, n_float_tokens=None, report=None):
+    wl = li.wl
+    T = wl.T
+    lay = O.Layer(li)
+    x, bias, tok, tab = upload_activations(li)
+    # --- routing -------------------------------------------------------------
+    ids_o, w_o, margin, _ = lay.route()
+    ids_g, w_g = layer.route(x, bias, tok, tab)
+    torch.cuda.synchronize()
+    ids_g = ids_g.cpu().numpy()
+    w_g = w_g.cpu().numpy().astype(np.float64)
+    near = margin < NEAR_TIE
+    ok = ~near
+    assert np.array_equal(ids_g[ok], ids_o[ok]), "router ids differ on non-tie tokens"
+    if ok.any():
+        assert_close(w_g[ok], w_o[ok], "topk_w")
+    # --- permutation on the oracle's ids (bit-exact) ---------------------------
+    ids_dev = torch.from_numpy(ids_o).cuda()
+    counts, offsets, sorted_slot, slot_pos = layer.permute(ids_dev)
+    c_o, off_o, ss_o, sp_o = O.permute(ids_o, wl.E)
+    torch.cuda.synchronize()
+    assert np.array_equal(counts.cpu().numpy(), c_o)
+    assert np.array_equal(offsets.cpu().numpy(), off_o)
+    S = T * wl.k
+    assert np.array_equal(sorted_slot.cpu().numpy()[:S], ss_o)
+    assert np.array_equal(slot_pos.cpu().numpy()[:S], sp_o)
+    # --- forward on the oracle's routing ---------------------------------------
+    w32 = w_o.astype(np.float32)
+    w_dev = torch.from_numpy(w32).cuda()
+    out = layer.forward(x, ids_dev, w_dev, offsets, sorted_slot, slot_pos)
+    torch.cuda.synchronize()
+    got = bf16_to_f64(out)
+    toks = sample_tokens(T, ids_o, n_float_tokens or T)
+    ref = lay.moe_tokens(toks, ids_o, w32.astype(np.float64), threads=host_threads())
+    rel, mabs = assert_close(got[toks], ref, f"{wl.name} out")
+    # --- end to end (GPU routing) on tokens whose routing is unambiguous ------
+    out2 = layer(x, bias, tok, tab)
+    torch.cuda.synchronize()
+    got2 = bf16_to_f64(out2)
+    e2e = toks[ok[toks]]
+    if e2e.size:
+        assert_close(got2[e2e], ref[ok[toks]], f"{wl.name} end-to-end")
+    if report is not None:
+        report.update(near_ties=int(near.sum()), rel_l2=rel, max_abs=mabs, tokens=len(toks))
+    return got, ref
+
+
+def test_tiny_layer_all_tokens():
+    li = IN.make_layer_inputs(IN.WORKLOADS["tiny"])
+    rep = {}
+    run_parity(li, _layer(li), report=rep)
+    print("tiny", rep)
+
+
+@pytest.mark.parametrize("T", [1, 7, 37, 300])
+def test_ragged_token_counts_multi_tile(T):
+    wl = IN.Workload("mid", T=T, H=1024, E=32, I=512, Is=256, bias_std=0.05, seed=11)
+    li = IN.make_layer_inputs(wl)
+    run_parity(li, _layer(li))
+
+
+def test_hash_routing_small():
+    wl = IN.Workload("hash_small", T=200, H=512, E=16, I=256, Is=256, routing="hash", vocab=1000,
+                     seed=5)
+    li = IN.make_layer_inputs(wl)
+    run_parity(li, _layer(li))
+
+
+def test_no_shared_expert_and_k1():
+    wl = IN.Workload("noshared", T=50, H=256, E=8, k=1, I=128, Is=0, seed=2)
+    li = IN.make_layer_inputs(wl)
+    run_parity(li, _layer(li))
+
+
+def test_all_tokens_on_one_expert_set():
+    wl = IN.Workload("skew", T=129, H=512, E=16, I=256, Is=256, seed=4)
+    li = IN.make_layer_inputs(wl)
+    layer = _layer(li)
+    ids = np.tile(np.array([[2, 3, 5, 7, 11, 13]], np.int32), (wl.T, 1))
+    w = np.full((wl.T, 6), 0.25, np.float32)
+    x, *_ = upload_activations(li)
+    ids_d = torch.from_numpy(ids).cuda()
+    _, offsets, ss, sp = layer.permute(ids_d)
+    out = layer.forward(x, ids_d, torch.from_numpy(w).cuda(), offsets, ss, sp)
+    torch.cuda.synchronize()
+    ref = O.Layer(li).moe_tokens(np.arange(wl.T), ids, w.astype(np.float64), threads=host_threads())
+    assert_close(bf16_to_f64(out), ref, "skew")
+
+
+def test_empty_batch():
+    wl = IN.Workload("empty", T=0, H=512, E=16, I=256, Is=256)
+    li = IN.make_layer_inputs(wl.with_T(4))
+    layer = _layer(li)
+    x = torch.empty((0, 512), dtype=torch.bfloat16, device="cuda")
+    bias = torch.zeros(16, device="cuda")
+    out = layer(x, bias)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 512)
+    assert not layer.buffers(0)["offsets"].any().item()
+
+
+def test_bad_ids_flagged_not_faulting():
+    import mxfp4_routed_expert_v4moe_b200 as V
+    wl = IN.Workload("bad", T=16, H=512, E=16, I=256, Is=256)
+    li = IN.make_layer_inputs(wl)
+    layer = _layer(li)
+    ws = layer.workspace(16)
+    assert V.v4moe_clear_device_status(ws) == 0
+    assert V.v4moe_read_device_status(ws) == V.V4MOE_OK
+    ids = np.zeros((16, 6), np.int32)
+    ids[:, :] = np.arange(6)
+    ids[3, 2] = 16      # out of range
+    ids[5, 0] = -1      # negative
+    layer.permute(torch.from_numpy(ids).cuda())
+    assert V.v4moe_read_device_status(ws) == V.V4MOE_ERR_DATA
+    V.v4moe_clear_device_status(ws)
+    assert V.v4moe_read_device_status(ws) == V.V4MOE_OK
+    # hash routing with a token id beyond the table
+    wlh = IN.Workload("badh", T=16, H=512, E=16, I=256, Is=256, routing="hash", vocab=50)
+    lih = IN.make_layer_inputs(wlh)
+    layh = _layer(lih)
+    x, _, tok, tab = upload_activations(lih)
+    tok[4] = 50
+    ids_g, w_g = layh.route(x, None, tok, tab)
+    assert V.v4moe_read_device_status(layh.workspace(16)) == V.V4MOE_ERR_DATA
+    assert float(w_g[4].abs().sum().item()) == 0.0
+
+
+@pytest.mark.parametrize("name,n_tok", [("decode_b1", None), ("decode_b64", None),
+                                        ("prefill_4096", 48), ("hash_16384", 48)])
+def test_full_size_workloads(name, n_tok, full_weights):
+    wl = IN.WORKLOADS[name]
+    li = IN.make_layer_inputs(wl, weights=full_weights)
+    rep = {}
+    run_parity(li, _layer(li), n_float_tokens=n_tok, report=rep)
+    print(name, rep)

@@ -318,3 +318,14 @@ def test_output_is_linear_in_routing_weights():
     a = lay.moe_tokens(np.arange(3), ids, w)
     b = lay.moe_tokens(np.arange(3), ids, 2.0 * w)
     assert np.allclose(b, 2.0 * a, rtol=1e-14, atol=0)
+
+
+def test_threaded_token_split_changes_nothing():
+    li = tiny_inputs(T=7, H=64, E=8, k=3, I=32, Is=32)
+    lay = O.Layer(li)
+    ids, w, _, _ = lay.route()
+    a = lay.moe_tokens(np.arange(7), ids, w, threads=1)
+    b = lay.moe_tokens(np.arange(7), ids, w, threads=3)
+    assert np.array_equal(a, b)
+    a2, h2, hs2 = lay.moe_tokens(np.array([6, 1]), ids, w, threads=2, want_h=True)
+    assert np.array_equal(a2, a[[6, 1]])
