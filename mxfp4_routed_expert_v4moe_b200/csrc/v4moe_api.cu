@@ -8,8 +8,6 @@
 
 namespace v4moe {
 
-cudaError_t launch_forward_simt(const ForwardArgs& a, cudaStream_t st);
-
 namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -154,7 +152,9 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x, const i
   a.y_slot = at<float>(ws, L.y_slot);
   a.hs = at<__nv_bfloat16>(ws, L.hs);
   a.ys = at<float>(ws, L.ys);
-  return launch_status(launch_forward_simt(a, static_cast<cudaStream_t>(stream)));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dec_supported(*cfg, T)) return launch_status(launch_forward_dec(a, st));
+  return launch_status(launch_forward_simt(a, st));
 }
 
 int32_t v4moe_read_device_status(const void* ws, void* stream) {

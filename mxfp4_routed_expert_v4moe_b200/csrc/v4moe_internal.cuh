@@ -90,6 +90,11 @@ struct ForwardArgs {
 
 cudaError_t launch_forward_simt(const ForwardArgs& a, cudaStream_t st);
 
+// Decode path (tensor-core weight streaming) for small token counts.
+constexpr int kDecodeMaxTokens = 64;
+bool dec_supported(const v4moe_config& c, int T);
+cudaError_t launch_forward_dec(const ForwardArgs& a, cudaStream_t st);
+
 // ---------------------------------------------------------------- device helpers
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
