@@ -130,6 +130,30 @@ int32_t v4moe_permute(const v4moe_config* cfg, int32_t T, const int32_t* topk_id
                       int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
                       int32_t* slot_pos, void* ws, size_t ws_bytes, void* stream);
 
+/* v4moe_permute without a workspace, for callers that cannot allocate device
+ * memory (the paper has no counterpart: this is a deployment variant).
+ * Some runtimes plan all device memory at start-up and forbid allocations
+ * afterwards, and some host code must not reach a device allocator at all
+ * (it may synchronise the device or fail under memory pressure). This entry
+ * point computes exactly what v4moe_permute computes, with the same arguments
+ * minus ws/ws_bytes; its scratch is a fixed array of about 256 KiB inside the
+ * library that every GPU loading the library holds until the process exits.
+ *  - Limits: T * top_k <= 65536 and n_experts <= 1024; larger sizes return
+ *    V4MOE_ERR_INVALID_ARG before anything is launched.
+ *  - It allocates nothing (no cudaMalloc/cudaFree, no allocating library
+ *    call). The first call on a device looks up the array's device address
+ *    with cudaGetSymbolAddress (once per device, with that device current);
+ *    make that first call before any stream capture.
+ *  - Every call shares the one array. Calls whose kernels may overlap on the
+ *    GPU (different streams, or several host threads) race on it and must be
+ *    serialised by the caller.
+ *  - Out-of-range ids are skipped as in v4moe_permute, but the device status
+ *    word is internal to the array (cleared at the start of each call) and
+ *    cannot be read back; use v4moe_permute when errors must be reported. */
+int32_t v4moe_permute_static(const v4moe_config* cfg, int32_t T, const int32_t* topk_ids,
+                             int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
+                             int32_t* slot_pos, void* stream);
+
 /* Expert computation and combine:
  *   out[t] = bf16( sum_j topk_w[t,j] * FFN_{topk_ids[t,j]}(x[t]) + FFN_shared(x[t]) )
  * with the clamped SwiGLU ("Checked in its code" row "SwiGLU feed-forward":

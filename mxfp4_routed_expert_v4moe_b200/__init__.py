@@ -29,7 +29,7 @@ V4MOE_ERR_TIMEOUT = 6
 EXPORTED = ("v4moe_workspace_bytes", "v4moe_route", "v4moe_permute", "v4moe_forward",
             "v4moe_read_device_status", "v4moe_clear_device_status", "v4moe_status_string",
             "v4moe_profile_enable", "v4moe_profile_reset", "v4moe_profile_read",
-            "v4moe_launch_count")
+            "v4moe_launch_count", "v4moe_permute_static")
 
 
 class V4moeError(RuntimeError):
@@ -72,6 +72,8 @@ def load(path: str | None = None):
             L.v4moe_route.restype = i32
             L.v4moe_permute.argtypes = [cfgp, i32, P, P, P, P, P, P, sz, P]
             L.v4moe_permute.restype = i32
+            L.v4moe_permute_static.argtypes = [cfgp, i32, P, P, P, P, P, P]
+            L.v4moe_permute_static.restype = i32
             L.v4moe_forward.argtypes = [cfgp, i32, P, P, P, P, P, P, ctypes.POINTER(v4moe_weights),
                                         P, P, sz, P]
             L.v4moe_forward.restype = i32
@@ -148,6 +150,15 @@ def v4moe_permute(cfg, T, topk_ids, counts, offsets, sorted_slot, slot_pos, ws, 
     return load().v4moe_permute(ctypes.byref(cfg), T, _ptr(topk_ids), _ptr(counts), _ptr(offsets),
                                 _ptr(sorted_slot), _ptr(slot_pos), _ptr(ws), ws_bytes,
                                 _stream(stream))
+
+
+def v4moe_permute_static(cfg, T, topk_ids, counts, offsets, sorted_slot, slot_pos,
+                         stream=None) -> int:
+    """v4moe_permute for callers that cannot allocate: no workspace argument;
+    scratch lives in a fixed array inside the library (see include/v4moe.h)."""
+    return load().v4moe_permute_static(ctypes.byref(cfg), T, _ptr(topk_ids), _ptr(counts),
+                                       _ptr(offsets), _ptr(sorted_slot), _ptr(slot_pos),
+                                       _stream(stream))
 
 
 def v4moe_forward(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, weights, out, ws,

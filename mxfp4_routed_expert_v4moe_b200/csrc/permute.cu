@@ -8,6 +8,9 @@
 // one CTA scans experts and chunk bases, then one warp per chunk scatters its
 // slots in order. Stability inside a chunk comes from walking the chunk in
 // slot order, 32 slots at a time, with __match_any_sync ranking equal ids.
+#include <mutex>
+#include <unordered_map>
+
 #include "launch.cuh"
 #include "v4moe_internal.cuh"
 
@@ -181,3 +184,91 @@ cudaError_t launch_permute(const v4moe_config& c, int T, const int32_t* topk_ids
 }
 
 }  // namespace v4moe
+
+// ---------------------------------------------------------------------------
+// Permutation without a caller workspace.
+//
+// Some callers cannot hand the library a device buffer: runtimes whose device
+// memory is planned once at start-up and may not grow afterwards, or host code
+// that must not reach a device allocator (which may synchronise the device or
+// fail under memory pressure). For them v4moe_permute_static keeps its scratch
+// in the fixed array below, which every GPU that loads this library holds
+// until the process exits.
+namespace v4moe {
+namespace {
+
+constexpr int kStaticMaxSlots = 1 << 16;                          // T * top_k limit
+constexpr int kStaticMaxChunks = kStaticMaxSlots / kPermChunk;    // 32
+constexpr int kStaticStatusWords = 64;                            // 256-byte status block
+constexpr size_t kStaticWords = kStaticStatusWords + size_t(2) * kStaticMaxChunks * 1024;
+
+// Layout: [status block][chunk counts][chunk bases]. In host code this name
+// only stands for the array; its device address comes from
+// cudaGetSymbolAddress.
+__device__ __align__(256) int32_t g_perm_scratch[kStaticWords];
+
+std::mutex g_scratch_mu;
+std::unordered_map<int, int32_t*> g_scratch_addr;  // device ordinal -> device address
+
+// Device address of g_perm_scratch on the current device (looked up once per
+// device, with that device current).
+int32_t* static_scratch(cudaError_t* err) {
+  int dev = -1;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  auto it = g_scratch_addr.find(dev);
+  if (it != g_scratch_addr.end()) return it->second;
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, g_perm_scratch);
+  if (*err != cudaSuccess) return nullptr;
+  g_scratch_addr.emplace(dev, static_cast<int32_t*>(p));
+  return static_cast<int32_t*>(p);
+}
+
+}  // namespace
+}  // namespace v4moe
+
+extern "C" int32_t v4moe_permute_static(const v4moe_config* cfg, int32_t T, const int32_t* topk_ids,
+                                        int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
+                                        int32_t* slot_pos, void* stream) {
+  using namespace v4moe;
+  if (!cfg || T < 0 || cfg->top_k < 1 || cfg->top_k > 8 || cfg->n_experts < cfg->top_k ||
+      cfg->n_experts > 1024)
+    return V4MOE_ERR_INVALID_ARG;
+  if (!counts || !offsets) return V4MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_ids || !sorted_slot || !slot_pos)) return V4MOE_ERR_INVALID_ARG;
+  if (int64_t(T) * cfg->top_k > kStaticMaxSlots) return V4MOE_ERR_INVALID_ARG;
+  int dev = -1, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return V4MOE_ERR_UNSUPPORTED_DEVICE;
+  }
+  if (major != 10 || minor != 0) return V4MOE_ERR_UNSUPPORTED_DEVICE;
+  cudaError_t err = cudaSuccess;
+  int32_t* base = static_scratch(&err);
+  if (!base) {
+    cudaGetLastError();
+    return V4MOE_ERR_LAUNCH;
+  }
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int S = T * cfg->top_k;
+  const int nchunks = S > 0 ? (S + kPermChunk - 1) / kPermChunk : 1;
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  int32_t* chunk_counts = base + kStaticStatusWords;
+  int32_t* chunk_base = chunk_counts + size_t(nchunks) * cfg->n_experts;
+  // The status word is the only scratch that accumulates; start it at zero.
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) {
+    cudaGetLastError();
+    return V4MOE_ERR_LAUNCH;
+  }
+  const cudaError_t e = launch_permute(*cfg, T, topk_ids, counts, offsets, sorted_slot, slot_pos,
+                                       chunk_counts, chunk_base, nchunks, status, st);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return V4MOE_ERR_LAUNCH;
+  }
+  return V4MOE_OK;
+}
