@@ -29,10 +29,13 @@
  *    device memory on the host, except v4moe_read_device_status (which
  *    synchronises the stream, for tests and debugging).
  *  - Scratch memory comes from the caller's workspace `ws` of `ws_bytes`
- *    bytes (see v4moe_workspace_bytes); it must be 256-byte aligned. The
- *    first bytes of the workspace hold a device status word that kernels set
- *    when they meet bad data (an out-of-range expert or token id, which they
- *    skip) or give up a bounded wait; read it with v4moe_read_device_status.
+ *    bytes (see v4moe_workspace_bytes); it must be 256-byte aligned and
+ *    zero-filled before its first use (every call leaves its first 256 bytes
+ *    in a state the next call accepts; v4moe_clear_device_status restores
+ *    them). Those bytes hold a device status word that kernels set when they
+ *    meet bad data (an out-of-range expert or token id, which they skip) or
+ *    give up a bounded wait; read it with v4moe_read_device_status. Calls
+ *    that share a workspace must not overlap on the GPU.
  *  - Return value: a V4MOE_* status code. Argument errors are detected on the
  *    host before anything is launched; data errors are visible only through
  *    the device status word.
@@ -80,7 +83,9 @@ typedef struct v4moe_config {
  *  w2_scales  [E, H, I/32] uint8   E8M0
  *  sh_w13     [2I_s, H] int8, sh_w13_scale [2I_s] fp32  (gate rows then up rows)
  *  sh_w2      [H, I_s]  int8, sh_w2_scale  [H] fp32
- * The shared-expert pointers may be NULL only when shared_inter == 0. */
+ * Code pointers and E8M0 scale pointers must be 16-byte aligned, fp32 scale
+ * pointers 4-byte aligned. The shared-expert pointers may be NULL only when
+ * shared_inter == 0. */
 typedef struct v4moe_weights {
   const uint8_t* w13_codes;
   const uint8_t* w13_scales;
@@ -167,6 +172,18 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x,
                       const int32_t* sorted_slot, const int32_t* slot_pos,
                       const v4moe_weights* weights, void* out, void* ws, size_t ws_bytes,
                       void* stream);
+
+/* The whole layer in one call: v4moe_route, v4moe_permute and v4moe_forward
+ * with the same arguments and results (routing outputs included). For small
+ * batches (T <= 8) routing, permutation and the activation layout run as a
+ * single fused kernel (its last CTA does the selection and the sort), and the
+ * expert kernels stream the shared expert's weights while routing is still
+ * being computed. */
+int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const void* gate,
+                    const float* bias, const int32_t* token_ids, const int32_t* tid2eid,
+                    const v4moe_weights* weights, int32_t* topk_ids, float* topk_w,
+                    int32_t* counts, int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos,
+                    void* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, reads the device status word of `ws` and returns
  * V4MOE_OK, V4MOE_ERR_DATA or V4MOE_ERR_TIMEOUT (or V4MOE_ERR_LAUNCH if the

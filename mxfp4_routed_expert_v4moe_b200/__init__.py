@@ -29,7 +29,7 @@ V4MOE_ERR_TIMEOUT = 6
 EXPORTED = ("v4moe_workspace_bytes", "v4moe_route", "v4moe_permute", "v4moe_forward",
             "v4moe_read_device_status", "v4moe_clear_device_status", "v4moe_status_string",
             "v4moe_profile_enable", "v4moe_profile_reset", "v4moe_profile_read",
-            "v4moe_launch_count", "v4moe_permute_static")
+            "v4moe_launch_count", "v4moe_permute_static", "v4moe_layer")
 
 
 class V4moeError(RuntimeError):
@@ -77,6 +77,9 @@ def load(path: str | None = None):
             L.v4moe_forward.argtypes = [cfgp, i32, P, P, P, P, P, P, ctypes.POINTER(v4moe_weights),
                                         P, P, sz, P]
             L.v4moe_forward.restype = i32
+            L.v4moe_layer.argtypes = [cfgp, i32, P, P, P, P, P, ctypes.POINTER(v4moe_weights), P, P, P, P,
+                                      P, P, P, P, sz, P]
+            L.v4moe_layer.restype = i32
             L.v4moe_read_device_status.argtypes = [P, P]
             L.v4moe_read_device_status.restype = i32
             L.v4moe_clear_device_status.argtypes = [P, P]
@@ -167,6 +170,14 @@ def v4moe_forward(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, w
                                 _ptr(offsets), _ptr(sorted_slot), _ptr(slot_pos),
                                 ctypes.byref(weights), _ptr(out), _ptr(ws), ws_bytes,
                                 _stream(stream))
+
+
+def v4moe_layer(cfg, T, x, gate, bias, token_ids, tid2eid, weights, topk_ids, topk_w, counts,
+                offsets, sorted_slot, slot_pos, out, ws, ws_bytes, stream=None) -> int:
+    return load().v4moe_layer(ctypes.byref(cfg), T, _ptr(x), _ptr(gate), _ptr(bias), _ptr(token_ids),
+                              _ptr(tid2eid), ctypes.byref(weights), _ptr(topk_ids), _ptr(topk_w),
+                              _ptr(counts), _ptr(offsets), _ptr(sorted_slot), _ptr(slot_pos),
+                              _ptr(out), _ptr(ws), ws_bytes, _stream(stream))
 
 
 def v4moe_read_device_status(ws, stream=None) -> int:

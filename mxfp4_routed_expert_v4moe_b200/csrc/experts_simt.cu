@@ -277,6 +277,13 @@ __global__ void __launch_bounds__(256) k_combine(int T, int H, int E, int k, con
 
 }  // namespace
 
+cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t st) {
+  const v4moe_config& c = a.c;
+  return launch_kernel("combine", k_combine, dim3(a.T), dim3(256), 0, st, false, a.T, c.hidden, c.n_experts,
+                       c.top_k, a.topk_ids, a.topk_w, a.slot_pos, (const float*)a.y_slot,
+                       (const float*)(c.shared_inter > 0 ? a.ys : nullptr), a.out);
+}
+
 cudaError_t launch_forward_simt(const ForwardArgs& a, cudaStream_t st) {
   const v4moe_config& c = a.c;
   if (a.T == 0) return cudaSuccess;

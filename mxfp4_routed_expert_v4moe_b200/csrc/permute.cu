@@ -12,40 +12,13 @@
 #include <unordered_map>
 
 #include "launch.cuh"
+#include "route_dev.cuh"
 #include "v4moe_internal.cuh"
 
 namespace v4moe {
 namespace {
 
 __device__ __forceinline__ bool id_ok(int e, int E) { return e >= 0 && e < E; }
-
-// Walks slots [s0, s1) in order with one warp; cursor[e] (shared) holds the
-// next output position of expert e and is advanced.
-__device__ __forceinline__ void warp_stable_scatter(const int32_t* __restrict__ ids, int s0, int s1,
-                                                    int E, int* cursor, int32_t* __restrict__ sorted_slot,
-                                                    int32_t* __restrict__ slot_pos) {
-  const int lane = threadIdx.x & 31;
-  for (int base = s0; base < s1; base += 32) {
-    const int s = base + lane;
-    int e = -1;
-    if (s < s1) {
-      e = ids[s];
-      if (!id_ok(e, E)) e = -1;
-    }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    int pos = 0;
-    if (e >= 0) pos = cursor[e] + rank;
-    __syncwarp();
-    if (e >= 0) {
-      const int leader = __ffs(peers) - 1;
-      if (lane == leader) cursor[e] += __popc(peers);
-      sorted_slot[pos] = s;
-      slot_pos[s] = pos;
-    }
-    __syncwarp();
-  }
-}
 
 // Exclusive scan of v over the block (blockDim.x == 1024, one value per
 // thread); returns the exclusive prefix, *total gets the sum.

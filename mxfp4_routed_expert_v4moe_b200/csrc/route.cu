@@ -16,6 +16,7 @@
 // Hash routing, one kernel (k_route_hash): one warp per token reads its
 // tid2eid row and computes only the k needed gate dot products.
 #include "launch.cuh"
+#include "route_dev.cuh"
 #include "v4moe_internal.cuh"
 
 namespace v4moe {
@@ -98,91 +99,13 @@ __global__ void __launch_bounds__(256) k_route_scores(int T, int H, int E,
   }
 }
 
-// Insertion sort of k <= 8 ids held identically by every lane.
-__device__ __forceinline__ void sort_ids(int* id, int k) {
-  for (int i = 1; i < 8; ++i) {
-    if (i >= k) break;
-    const int v = id[i];
-    int j = i - 1;
-    while (j >= 0 && id[j] > v) {
-      id[j + 1] = id[j];
-      --j;
-    }
-    id[j + 1] = v;
-  }
-}
-
 __global__ void __launch_bounds__(kSelectWarps * 32) k_route_select(
-    int T, int E, int k, float routed_scale, const float* __restrict__ scores,
-    const float* __restrict__ bias, int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int T, int E, int k, float routed_scale, const float* scores, const float* __restrict__ bias,
+    int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
+  const int warp = threadIdx.x >> 5;
   const int t = blockIdx.x * kSelectWarps + warp;
   if (t >= T) return;
-  const float* s = scores + size_t(t) * E;
-  const int nper = (E + 31) / 32;
-  float b[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    float v = -INFINITY;
-    if (i < nper && e < E) {
-      v = s[e] + bias[e];
-      if (v != v) v = -INFINITY;  // NaN never wins
-    }
-    b[i] = v;
-  }
-  uint32_t taken = 0;
-  int id[8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    if (r >= k) {
-      id[r] = 0x7fffffff;
-      continue;
-    }
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int e = lane + 32 * i;
-      if (i < nper && e < E && !((taken >> i) & 1u)) {
-        if (b[i] > bv || be == 0x7fffffff) {
-          bv = b[i];
-          be = e;
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    id[r] = be;
-  }
-  sort_ids(id, k);
-  float sum = 0.0f;
-  float sv[8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    sv[r] = (r < k) ? s[id[r]] : 0.0f;
-    sum += sv[r];
-  }
-  if (lane < k) {
-    float myv = 0.0f;
-    int myid = 0;
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r == lane) {
-        myv = sv[r];
-        myid = id[r];
-      }
-    topk_ids[size_t(t) * k + lane] = myid;
-    topk_w[size_t(t) * k + lane] = routed_scale * (myv / sum);
-  }
+  select_learned_warp(t, E, k, routed_scale, scores + size_t(t) * E, bias, topk_ids, topk_w);
 }
 
 __global__ void __launch_bounds__(kSelectWarps * 32) k_route_hash(

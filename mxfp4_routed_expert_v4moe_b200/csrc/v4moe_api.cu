@@ -112,29 +112,30 @@ int32_t v4moe_permute(const v4moe_config* cfg, int32_t T, const int32_t* topk_id
                                       static_cast<cudaStream_t>(stream)));
 }
 
-int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x, const int32_t* topk_ids,
-                      const float* topk_w, const int32_t* offsets, const int32_t* sorted_slot,
-                      const int32_t* slot_pos, const v4moe_weights* weights, void* out, void* ws,
-                      size_t ws_bytes, void* stream) {
-  if (!config_ok(cfg) || T < 0 || !weights) return V4MOE_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace v4moe {
+namespace {
+
+int32_t check_weights(const v4moe_config* cfg, const v4moe_weights* weights) {
+  if (!weights) return V4MOE_ERR_INVALID_ARG;
   const v4moe_weights& w = *weights;
   if (!w.w13_codes || !w.w13_scales || !w.w2_codes || !w.w2_scales) return V4MOE_ERR_INVALID_ARG;
-  if (!aligned(w.w13_codes, 16) || !aligned(w.w2_codes, 16) || !aligned(w.w13_scales, 4) ||
-      !aligned(w.w2_scales, 4))
+  if (!aligned(w.w13_codes, 16) || !aligned(w.w2_codes, 16) || !aligned(w.w13_scales, 16) ||
+      !aligned(w.w2_scales, 16))
     return V4MOE_ERR_INVALID_ARG;
   if (cfg->shared_inter > 0) {
     if (!w.sh_w13 || !w.sh_w13_scale || !w.sh_w2 || !w.sh_w2_scale) return V4MOE_ERR_INVALID_ARG;
-    if (!aligned(w.sh_w13, 16) || !aligned(w.sh_w2, 16)) return V4MOE_ERR_INVALID_ARG;
+    if (!aligned(w.sh_w13, 16) || !aligned(w.sh_w2, 16) || !aligned(w.sh_w13_scale, 4) ||
+        !aligned(w.sh_w2_scale, 4))
+      return V4MOE_ERR_INVALID_ARG;
   }
-  if (!offsets) return V4MOE_ERR_INVALID_ARG;
-  if (T > 0) {
-    if (!x || !topk_ids || !topk_w || !sorted_slot || !slot_pos || !out) return V4MOE_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(out, 16)) return V4MOE_ERR_INVALID_ARG;
-    if (x == out) return V4MOE_ERR_INVALID_ARG;
-  }
-  if (int32_t r = check_ws(cfg, T, ws, ws_bytes)) return r;
-  if (int32_t r = check_device()) return r;
-  if (T == 0) return V4MOE_OK;
+  return V4MOE_OK;
+}
+
+ForwardArgs forward_args(const v4moe_config* cfg, int32_t T, const void* x, const int32_t* topk_ids,
+                         const float* topk_w, const int32_t* offsets, const int32_t* sorted_slot,
+                         const int32_t* slot_pos, const v4moe_weights* weights, void* out, void* ws) {
   const WsLayout L = ws_layout(*cfg, T);
   ForwardArgs a;
   a.c = *cfg;
@@ -145,16 +146,88 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x, const i
   a.offsets = offsets;
   a.sorted_slot = sorted_slot;
   a.slot_pos = slot_pos;
-  a.w = w;
+  a.w = *weights;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.status = at<uint32_t>(ws, L.status);
   a.h = at<__nv_bfloat16>(ws, L.h);
   a.y_slot = at<float>(ws, L.y_slot);
   a.hs = at<__nv_bfloat16>(ws, L.hs);
   a.ys = at<float>(ws, L.ys);
+  return a;
+}
+
+}  // namespace
+}  // namespace v4moe
+
+extern "C" {
+
+int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x, const int32_t* topk_ids,
+                      const float* topk_w, const int32_t* offsets, const int32_t* sorted_slot,
+                      const int32_t* slot_pos, const v4moe_weights* weights, void* out, void* ws,
+                      size_t ws_bytes, void* stream) {
+  if (!config_ok(cfg) || T < 0) return V4MOE_ERR_INVALID_ARG;
+  if (int32_t r = check_weights(cfg, weights)) return r;
+  if (!offsets) return V4MOE_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!x || !topk_ids || !topk_w || !sorted_slot || !slot_pos || !out) return V4MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16)) return V4MOE_ERR_INVALID_ARG;
+    if (x == out) return V4MOE_ERR_INVALID_ARG;
+  }
+  if (int32_t r = check_ws(cfg, T, ws, ws_bytes)) return r;
+  if (int32_t r = check_device()) return r;
+  if (T == 0) return V4MOE_OK;
+  const WsLayout L = ws_layout(*cfg, T);
+  const ForwardArgs a = forward_args(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, weights, out, ws);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dec_supported(*cfg, T)) return launch_status(launch_forward_dec(a, st));
-  return launch_status(launch_forward_simt(a, st));
+  if (dec_supported(*cfg, T)) {
+    __half* xlog = at<__half>(ws, L.xlog);
+    int* sigma = at<int>(ws, L.sigma);
+    if (cudaError_t e = launch_dec_xlog(*cfg, T, a.x, xlog, sigma, st)) return launch_status(e);
+    return launch_status(launch_forward_dec(a, xlog, sigma, st));
+  }
+  return launch_status(launch_forward_tc(a, at<__half>(ws, L.xlog), at<int>(ws, L.sigma), at<char>(ws, L.tc), st));
+}
+
+int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const void* gate, const float* bias,
+                    const int32_t* token_ids, const int32_t* tid2eid, const v4moe_weights* weights,
+                    int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
+                    int32_t* slot_pos, void* out, void* ws, size_t ws_bytes, void* stream) {
+  if (!config_ok(cfg) || T < 0) return V4MOE_ERR_INVALID_ARG;
+  if (int32_t r = check_weights(cfg, weights)) return r;
+  const bool hash = token_ids != nullptr || tid2eid != nullptr;
+  if (hash && (bias || !token_ids || !tid2eid || cfg->vocab <= 0)) return V4MOE_ERR_INVALID_ARG;
+  if (!hash && !bias) return V4MOE_ERR_INVALID_ARG;
+  if (!counts || !offsets) return V4MOE_ERR_INVALID_ARG;
+  if (T > 0) {
+    if (!x || !gate || !topk_ids || !topk_w || !sorted_slot || !slot_pos || !out) return V4MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(gate, 16) || !aligned(out, 16) || x == out) return V4MOE_ERR_INVALID_ARG;
+  }
+  if (int64_t(T) * cfg->top_k > 0x7fffffff / 2) return V4MOE_ERR_INVALID_ARG;
+  if (int32_t r = check_ws(cfg, T, ws, ws_bytes)) return r;
+  if (int32_t r = check_device()) return r;
+  // an empty batch still reports empty counts and offsets
+  if (T == 0) return v4moe_permute(cfg, 0, topk_ids, counts, offsets, sorted_slot, slot_pos, ws, ws_bytes, stream);
+  const WsLayout L = ws_layout(*cfg, T);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (dec_supported(*cfg, T)) {
+    __half* xlog = at<__half>(ws, L.xlog);
+    int* sigma = at<int>(ws, L.sigma);
+    uint32_t* status = at<uint32_t>(ws, L.status);
+    if (cudaError_t e = launch_dec_prep(*cfg, T, xb, static_cast<const __nv_bfloat16*>(gate), bias, token_ids,
+                                        tid2eid, topk_ids, topk_w, counts, offsets, sorted_slot, slot_pos,
+                                        at<float>(ws, L.scores), xlog, sigma, status,
+                                        reinterpret_cast<unsigned*>(status + kTicketWord), st))
+      return launch_status(e);
+    const ForwardArgs a = forward_args(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, weights, out, ws);
+    return launch_status(launch_forward_dec(a, xlog, sigma, st));
+  }
+  if (int32_t r = v4moe_route(cfg, T, x, gate, bias, token_ids, tid2eid, topk_ids, topk_w, ws, ws_bytes, stream))
+    return r;
+  if (int32_t r = v4moe_permute(cfg, T, topk_ids, counts, offsets, sorted_slot, slot_pos, ws, ws_bytes, stream))
+    return r;
+  return v4moe_forward(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, weights, out, ws, ws_bytes,
+                       stream);
 }
 
 int32_t v4moe_read_device_status(const void* ws, void* stream) {

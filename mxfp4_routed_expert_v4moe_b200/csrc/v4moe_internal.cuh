@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -9,7 +10,10 @@
 
 namespace v4moe {
 
-// Device status word bits (first 4 bytes of the workspace).
+// Status block (first 256 bytes of the workspace): word 0 is the device
+// status word, word 1 the ticket of the fused decode preparation kernel.
+constexpr size_t kTicketWord = 1;
+// Device status word bits.
 constexpr uint32_t kStatusBadExpertId = 1u << 0;
 constexpr uint32_t kStatusBadTokenId = 1u << 1;
 constexpr uint32_t kStatusTimeout = 1u << 2;
@@ -19,6 +23,8 @@ inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a
 
 // Slots per chunk of the multi-CTA permutation.
 constexpr int kPermChunk = 2048;
+
+size_t tc_extra_bytes(const v4moe_config& c, int64_t T);
 
 // Workspace carve-up for T tokens. All offsets are 256-byte aligned.
 struct WsLayout {
@@ -30,6 +36,9 @@ struct WsLayout {
   size_t y_slot = 0;        // [T*k, H] fp32 routed expert outputs (sorted order)
   size_t hs = 0;            // [T, I_s] bf16 shared intermediates
   size_t ys = 0;            // [T, H] fp32 shared expert outputs
+  size_t xlog = 0;          // [T, H] f16 activations in the decode layout
+  size_t sigma = 0;         // [T] int32 per-token power-of-two exponents
+  size_t tc = 0;            // tensor-core path: activations in slot order + tile lists
   size_t total = 0;
   int nchunks = 0;
 };
@@ -53,6 +62,9 @@ inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
   L.y_slot = take(size_t(S) * c.hidden * 4);
   L.hs = take(size_t(T) * (c.shared_inter > 0 ? c.shared_inter : 0) * 2);
   L.ys = take(size_t(T) * c.hidden * 4);
+  L.xlog = take(size_t(T) * c.hidden * 2);
+  L.sigma = take(size_t(T) * 4);
+  L.tc = take(tc_extra_bytes(c, T));
   L.total = off;
   return L;
 }
@@ -89,11 +101,21 @@ struct ForwardArgs {
 };
 
 cudaError_t launch_forward_simt(const ForwardArgs& a, cudaStream_t st);
+cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t st);
+// Tensor-core path (tcgen05 grouped GEMMs) for larger token counts.
+cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, cudaStream_t st);
 
 // Decode path (tensor-core weight streaming) for small token counts.
-constexpr int kDecodeMaxTokens = 64;
+constexpr int kDecodeMaxTokens = 8;
 bool dec_supported(const v4moe_config& c, int T);
-cudaError_t launch_forward_dec(const ForwardArgs& a, cudaStream_t st);
+cudaError_t launch_forward_dec(const ForwardArgs& a, const __half* xlog, const int* sigma, cudaStream_t st);
+cudaError_t launch_dec_xlog(const v4moe_config& c, int T, const __nv_bfloat16* x, __half* xlog, int* sigma,
+                            cudaStream_t st);
+cudaError_t launch_dec_prep(const v4moe_config& c, int T, const __nv_bfloat16* x, const __nv_bfloat16* gate,
+                            const float* bias, const int32_t* token_ids, const int32_t* tid2eid,
+                            int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets,
+                            int32_t* sorted_slot, int32_t* slot_pos, float* scores, __half* xlog, int* sigma,
+                            uint32_t* status, unsigned* ticket, cudaStream_t st);
 
 // ---------------------------------------------------------------- device helpers
 

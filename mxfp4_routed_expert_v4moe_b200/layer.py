@@ -8,8 +8,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (check, make_config, make_weights, v4moe_forward, v4moe_permute, v4moe_route,
-               v4moe_workspace_bytes)
+from . import (check, make_config, make_weights, v4moe_forward, v4moe_layer, v4moe_permute,
+               v4moe_route, v4moe_workspace_bytes)
 
 
 class MoELayer:
@@ -96,6 +96,12 @@ class MoELayer:
         return out
 
     def __call__(self, x, bias=None, token_ids=None, tid2eid=None, out=None, stream=None):
-        ids, w = self.route(x, bias, token_ids, tid2eid, stream)
-        _, offsets, sorted_slot, slot_pos = self.permute(ids, stream)
-        return self.forward(x, ids, w, offsets, sorted_slot, slot_pos, out, stream)
+        """The whole layer through v4moe_layer (routing outputs kept in buffers(T))."""
+        T = x.shape[0]
+        b = self.buffers(T)
+        ws = self.workspace(T)
+        out = b["out"] if out is None else out
+        check(v4moe_layer(self.cfg, T, x, self.gate, bias, token_ids, tid2eid, self.weights,
+                          b["topk_ids"], b["topk_w"], b["counts"], b["offsets"], b["sorted_slot"],
+                          b["slot_pos"], out, ws, ws.numel(), stream), "v4moe_layer")
+        return out

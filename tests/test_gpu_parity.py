@@ -87,15 +87,17 @@ def test_ragged_token_counts_multi_tile(T):
     run_parity(li, _layer(li))
 
 
-def test_hash_routing_small():
-    wl = IN.Workload("hash_small", T=200, H=512, E=16, I=256, Is=256, routing="hash", vocab=1000,
+@pytest.mark.parametrize("T", [5, 200])
+def test_hash_routing_small(T):
+    wl = IN.Workload("hash_small", T=T, H=512, E=16, I=256, Is=256, routing="hash", vocab=1000,
                      seed=5)
     li = IN.make_layer_inputs(wl)
     run_parity(li, _layer(li))
 
 
-def test_no_shared_expert_and_k1():
-    wl = IN.Workload("noshared", T=50, H=256, E=8, k=1, I=128, Is=0, seed=2)
+@pytest.mark.parametrize("T", [3, 50])
+def test_no_shared_expert_and_k1(T):
+    wl = IN.Workload("noshared", T=T, H=256, E=8, k=1, I=128, Is=0, seed=2)
     li = IN.make_layer_inputs(wl)
     run_parity(li, _layer(li))
 
