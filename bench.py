@@ -4,8 +4,9 @@ int8 shared expert) on B200: prints ONE JSON line.
 
 A step is one pass of the whole layer -- route, permute, forward -- over one
 synthetic batch of the chosen workload (default: the full-size layer at decode
-batch 1). Inputs are resident in HBM when timing starts; L2 is flushed
-(512 MiB write) between timed steps; every step is timed with CUDA events on
+batch 1). Inputs are resident in HBM when timing starts; between timed steps
+L2 is flushed (512 MiB write, then a 256 MiB read so that no dirty lines are
+left for the next step to write back); every step is timed with CUDA events on
 the launch stream and the sum over steps is taken, max over ranks.
 
 Multi-GPU: replicas only (one process per GPU, each runs its own batch; no
@@ -33,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s"
 L2_FLUSH_BYTES = 512 << 20
+L2_CLEAN_BYTES = 256 << 20
 
 
 def parse():
@@ -271,6 +273,13 @@ def main():
     tab = None if li.tid2eid is None else torch.from_numpy(li.tid2eid).to(dev)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(L2_CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2(i):
+        # Write a buffer larger than L2, then read another one: the timed step
+        # starts with no useful data in L2 and no dirty lines left to write back.
+        flush.fill_(i & 0xFF)
+        clean.sum()
 
     def step():
         return layer(x, bias, tok, tab)
@@ -297,7 +306,7 @@ def main():
     torch.cuda.synchronize(dev)
     launches0 = V.v4moe_launch_count()
     for i in range(args.steps):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         evs[i][0].record(stream)
         step()
         evs[i][1].record(stream)
@@ -316,7 +325,7 @@ def main():
     e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     for i in range(args.steps):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         e2e_evs[i][0].record(stream)
         x_dev.copy_(x_host, non_blocking=True)
         if tok_dev is not None:
@@ -332,7 +341,7 @@ def main():
     V.v4moe_profile_reset()
     V.v4moe_profile_enable(True)
     for i in range(args.steps):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         step()
     torch.cuda.synchronize(dev)
     prof = V.v4moe_profile_read()
@@ -376,7 +385,7 @@ def main():
             "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
                        "shared_inter": wl.Is, "routing": wl.routing, "global_batch": wl.T * world,
                        "parallelism": f"replicas{world}", "experts_hit": acc["n_hit"],
-                       "l2": "flushed between timed steps (512 MiB write)",
+                       "l2": "flushed between timed steps (512 MiB write, then 256 MiB read)",
                        "weights": "MXFP4 routed (E2M1 + E8M0/32), int8 shared, bf16 gate"},
             "layer_roofline": {"algorithmic_bytes": acc["step_bytes"],
                                "algorithmic_flops": acc["step_flops"],

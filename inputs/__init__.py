@@ -202,6 +202,12 @@ WORKLOADS = {
                              notes="full-size layer, prefill 4096 tokens, near-uniform load"),
     "hash_16384": Workload("hash_16384", T=16384, routing="hash", bias_std=0.0,
                            notes="hash-routed layer, Zipf(1.1) token ids, skewed expert load"),
+    # Smaller cases of the same kernels for profiler captures (64 experts keep
+    # the weights under 1 GB; per-expert token counts match the full cases).
+    "decode_b1_e64": Workload("decode_b1_e64", T=1, E=64,
+                              notes="decode batch 1 with 64 experts (profiling size)"),
+    "prefill_1024_e64": Workload("prefill_1024_e64", T=1024, E=64,
+                                 notes="prefill, ~96 tokens per expert, 64 experts (profiling size)"),
 }
 WORKLOAD_ORDER = ["tiny", "decode_b1", "decode_b64", "prefill_4096", "hash_16384"]
 

@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256) k_dec_prep(PrepParams P) {
       select_hash_warp(t, E, P.k, P.vocab, P.routed_scale, s, P.token_ids, P.tid2eid, P.topk_ids, P.topk_w,
                        P.status);
     else
-      select_learned_warp(t, E, P.k, P.routed_scale, s, P.bias, P.topk_ids, P.topk_w);
+      select_learned<true>(t, E, P.k, P.routed_scale, s, P.bias, P.topk_ids, P.topk_w);
   }
   __syncthreads();
   cta_permute(T * P.k, E, P.topk_ids, P.counts, P.offsets, P.sorted_slot, P.slot_pos, P.status, cnt, cursor);

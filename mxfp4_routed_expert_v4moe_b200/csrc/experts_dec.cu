@@ -82,6 +82,8 @@ __host__ __device__ inline int stage_size(int fmt, int K) {
   return kTileRows * tile_stride(fmt, K) + (fmt == kMx ? kTileRows * (K / 32) : 0);
 }
 
+__device__ __forceinline__ size_t umin_(size_t a, size_t b) { return a < b ? a : b; }
+
 __device__ __forceinline__ float pow2f(int e) {
   e = max(-126, min(127, e));
   return __int_as_float((e + 127) << 23);
@@ -279,6 +281,60 @@ __global__ void __launch_bounds__(kDThreads) k_dec_w13(DecParams P) {
   };
   if (it0 < it1 && threadIdx.x == 0)
     for (int s = 0; s < P.stages && it0 + s < it1; ++s) issue(it0 + s, s);
+  // Ask for every later tile of this CTA now, into L2: the whole weight stream
+  // of the kernel is then in flight at once and the ring's copies hit L2.
+  if (warp == 1) {
+    for (int it = it0 + P.stages + lane; it < it1; it += 32) {
+      const int grp = item_group(it);
+      const int j0 = (it % blk) * 8;
+      if (shared_cta) {
+        const uint8_t* b = reinterpret_cast<const uint8_t*>(P.sh13);
+        prefetch_l2_bulk(b + size_t(j0) * H, uint32_t(8 * H));
+        prefetch_l2_bulk(b + size_t(Ig + j0) * H, uint32_t(8 * H));
+      } else {
+        const uint8_t* b = P.w13_codes + size_t(grp) * 2 * P.I * (H / 2);
+        const uint8_t* sc = P.w13_scales + size_t(grp) * 2 * P.I * (H / 32);
+        prefetch_l2_bulk(b + size_t(j0) * (H / 2), uint32_t(8 * (H / 2)));
+        prefetch_l2_bulk(b + size_t(Ig + j0) * (H / 2), uint32_t(8 * (H / 2)));
+        prefetch_l2_bulk(sc + size_t(j0) * (H / 32), uint32_t(8 * (H / 32)));
+        prefetch_l2_bulk(sc + size_t(Ig + j0) * (H / 32), uint32_t(8 * (H / 32)));
+      }
+    }
+  }
+  // The down projection of the same experts streams next: start moving its
+  // weights into L2 while this kernel runs (the routed CTAs split the hit
+  // experts' W2 blocks; the shared CTAs split the shared expert's).
+  if (warp == 2 && lane == 0) {
+    const int nctas = shared_cta ? P.n_shared_ctas : int(gridDim.x) - P.n_shared_ctas;
+    const int me = shared_cta ? int(blockIdx.x) : int(blockIdx.x) - P.n_shared_ctas;
+    if (shared_cta) {
+      const size_t total = size_t(H) * P.Is;
+      const size_t per = (total / nctas + 15) / 16 * 16;
+      const size_t a = size_t(me) * per;
+      if (a < total) prefetch_l2_range(reinterpret_cast<const uint8_t*>(P.sh2) + a, umin_(per, total - a));
+    } else if (n_routed > 0) {
+      const size_t codes = size_t(H) * (P.I / 2), scl = size_t(H) * (P.I / 32);
+      const size_t per_e = codes + scl;
+      const size_t total = per_e * n_routed;
+      const size_t per = (total / nctas + 15) / 16 * 16;
+      size_t a = size_t(me) * per;
+      const size_t b = umin_(total, a + per);
+      while (a < b) {
+        const int li = int(a / per_e);
+        size_t off = a - size_t(li) * per_e;
+        const size_t n = umin_(b - a, per_e - off);
+        const int e = list[li];
+        if (off < codes) {
+          const size_t nc = umin_(n, codes - off);
+          prefetch_l2_range(P.w2_codes + size_t(e) * codes + off, nc);
+          if (n > nc) prefetch_l2_range(P.w2_scales + size_t(e) * scl, n - nc);
+        } else {
+          prefetch_l2_range(P.w2_scales + size_t(e) * scl + (off - codes), n);
+        }
+        a += n;
+      }
+    }
+  }
   if (shared_cta) pdl_wait();  // the activations come from the preparation kernel
   if (it0 >= it1) return;
 

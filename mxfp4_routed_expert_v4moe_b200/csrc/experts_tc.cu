@@ -47,7 +47,7 @@ constexpr int BM = 128;            // weight rows per tile
 constexpr int BK = 64;             // K per stage (one 128-byte swizzle atom of f16)
 constexpr int BN = 128;            // max tokens per tile
 constexpr int kStages = 5;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;   // 16 warps: TMA, MMA, 2 idle, 4 epilogue, 8 dequantiser
 constexpr uint32_t kTries = 1u << 21;
 
 enum { kW13 = 0, kW2 = 1 };
@@ -78,6 +78,10 @@ struct TcParams {
   const int* sigma;                 // [T] token exponents of the f16 activations
   const TcTile* tiles;
   const int* ntiles;
+  const uint8_t* w_codes;           // routed codes (w13 or w2), for L2 prefetch
+  const uint8_t* sh_codes;          // shared int8 weights, for L2 prefetch
+  const __half* b_routed;           // activations of routed groups (x in slot order, or h)
+  const __half* b_shared;           // activations of the shared expert (x, or hs)
   const uint8_t* w_scales;          // routed E8M0 scales (w13 or w2)
   const float* sh_scale;            // shared expert fp32 row scales
   __half* h;                        // w13 out: [S, I]
@@ -184,12 +188,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&B.full_b[s], 1);
       mbar_init(&B.full_c[s], 1);
-      mbar_init(&B.full_a[s], 128);
+      mbar_init(&B.full_a[s], 8);  // one arrival per dequantiser warp
       mbar_init(&B.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&B.acc_full[b], 1);
-      mbar_init(&B.acc_empty[b], 128);
+      mbar_init(&B.acc_empty[b], 4);  // one arrival per epilogue warp
     }
     mbar_init(&B.done, 1);
     B.abort = 0;
@@ -220,6 +224,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const void* tmB = g.shared ? static_cast<const void*>(&tmB_s) : static_cast<const void*>(&tmB_r);
       const void* tmC = g.shared ? static_cast<const void*>(&tmC_s) : static_cast<const void*>(&tmC_r);
       const int cb = g.shared ? 64 : 32;  // code bytes per row per chunk
+      // Move the next tile's weights (and its activations, when they change)
+      // towards L2 now, so that its TMA loads do not wait on DRAM.
+      const int tn = ti + int(gridDim.x);
+      if (tn < ntiles) {
+        const TcTile t2 = P.tiles[tn];
+        const TileGeo g2 = geo(P, t2);
+        const size_t rb = g2.shared ? size_t(g2.K) : size_t(g2.K / 2);
+        const uint8_t* wb = g2.shared ? P.sh_codes : P.w_codes;
+        prefetch_l2_range(wb + size_t(g2.crow0) * rb, 64 * rb);
+        prefetch_l2_range(wb + size_t(g2.crow1) * rb, 64 * rb);
+        if (!g2.shared) {
+          const size_t G = size_t(g2.K / 32);
+          prefetch_l2_range(P.w_scales + size_t(g2.srow0) * G, 64 * G);
+          prefetch_l2_range(P.w_scales + size_t(g2.srow1) * G, 64 * G);
+        }
+        if (t2.grp != t.grp || t2.n0 != t.n0) {
+          const __half* bb = g2.shared ? P.b_shared : P.b_routed;
+          prefetch_l2_range(bb + size_t(g2.brow0) * g2.K, size_t(t2.n) * g2.K * 2);
+        }
+      }
       for (int c = 0; c < g.nk; ++c, ++gc) {
         const int s = gc % kStages;
         const uint32_t u = gc / kStages;
@@ -280,7 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait_bounded(&B.done, 0, kTries);
   } else if (warp >= 8) {
     // ------------------------------------------------------------ dequantisers
-    const int r = threadIdx.x - 256;  // tile row
+    const int dq = threadIdx.x - 256;
+    const int r = dq >> 1;   // tile row
+    const int hf = dq & 1;   // half of the 64-element chunk: elements [32 hf, 32 hf + 32)
     uint32_t gc = 0;
     bool ok = true;
     for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
@@ -312,32 +338,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const char* cs = smem + kOffC + s * kCStage;
-        uint32_t w[32];
+        uint32_t w[16];
         if (!g.shared) {
-          const uint4 q0 = *reinterpret_cast<const uint4*>(cs + r * 32);
-          const uint4 q1 = *reinterpret_cast<const uint4*>(cs + r * 32 + 16);
-          uint32_t sp;  // scale bytes of groups 2c, 2c+1
+          const uint4 q = *reinterpret_cast<const uint4*>(cs + r * 32 + hf * 16);
+          uint32_t e8;  // scale byte of group 2c + hf
           if (vec) {
             const uint32_t wv = (c & 4) ? ((c & 2) ? win.w : win.z) : ((c & 2) ? win.y : win.x);
-            sp = (wv >> ((c & 1) * 16)) & 0xFFFFu;
+            e8 = (wv >> ((c & 1) * 16 + hf * 8)) & 0xFFu;
           } else {
-            sp = __ldg(reinterpret_cast<const uint16_t*>(srow) + c);
+            e8 = __ldg(srow + 2 * c + hf);
           }
-          const uint32_t s0 = f16_pow2_bits(int(sp & 0xFF) - xmax + 13) * 0x10001u;
-          const uint32_t s1 = f16_pow2_bits(int(sp >> 8) - xmax + 13) * 0x10001u;
-          const uint32_t q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+          const uint32_t sc = f16_pow2_bits(int(e8) - xmax + 13) * 0x10001u;
+          const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
+          for (int i = 0; i < 4; ++i) {
             uint32_t f[4];
-            e2m1x8_to_f16x2(q[i], f);
-            const uint32_t sc = i < 4 ? s0 : s1;
+            e2m1x8_to_f16x2(qq[i], f);
 #pragma unroll
             for (int j = 0; j < 4; ++j) w[4 * i + j] = hmul2_u32(f[j], sc);
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 q = *reinterpret_cast<const uint4*>(cs + r * 64 + 16 * i);
+          for (int i = 0; i < 2; ++i) {
+            const uint4 q = *reinterpret_cast<const uint4*>(cs + r * 64 + hf * 32 + 16 * i);
             s8x4_to_f16x2(q.x, w[8 * i + 0], w[8 * i + 1]);
             s8x4_to_f16x2(q.y, w[8 * i + 2], w[8 * i + 3]);
             s8x4_to_f16x2(q.z, w[8 * i + 4], w[8 * i + 5]);
@@ -346,11 +369,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         char* as = smem + kOffA + s * kAStage + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4*>(as + ((j ^ (r & 7)) << 4)) =
+        for (int j = 0; j < 4; ++j) {
+          const int ch = 4 * hf + j;  // 16-byte chunk within the row
+          *reinterpret_cast<uint4*>(as + ((ch ^ (r & 7)) << 4)) =
               make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive(&B.full_a[s]);
+        }
+        fence_proxy_async_smem();  // make this thread's generic-proxy writes visible to the MMA
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.full_a[s]);
       }
     }
   } else if (warp >= 4) {
@@ -425,7 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&B.acc_empty[b]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.acc_empty[b]);
     }
   }
   tc_fence_before();
@@ -485,37 +512,68 @@ __global__ void __launch_bounds__(256) k_tc_gather(int T, int H, int E, int k, c
   }
 }
 
-// Tile lists of both GEMMs (one CTA): per group (routed experts in id order,
-// then the shared expert), token tiles of <= BN, times the row blocks.
+// Tile lists of both GEMMs (one CTA, one group per thread): per group
+// (routed experts in id order, then the shared expert), token tiles of <= BN,
+// times the row blocks (64 channels for w13, 128 output rows for w2). The
+// groups' tile counts are prefix-summed across the block.
+__device__ __forceinline__ int block_excl_scan_1024(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = warp_tot[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    warp_tot[lane] = wi - w;
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  return warp_tot[warp] + incl - v;
+}
+
 __global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, int Is, const int32_t* __restrict__ offsets,
                                                    TcTile* __restrict__ t13, int* __restrict__ n13, TcTile* __restrict__ t2,
                                                    int* __restrict__ n2) {
-  __shared__ int base13[1026], base2[1026];
-  const int G = E + (Is > 0 ? 1 : 0);
-  auto ntok = [&](int g) { return g < E ? offsets[g + 1] - offsets[g] : T; };
-  if (threadIdx.x == 0) {
-    int a = 0, b = 0;
-    for (int g = 0; g < G; ++g) {
-      const int tt = (ntok(g) + BN - 1) / BN;
-      base13[g] = a;
-      base2[g] = b;
-      a += tt * ((g < E ? I : Is) / 64);
-      b += tt * (H / 128);
+  __shared__ int wt13[32], wt2[32];
+  __shared__ int tot13, tot2;
+  const int G = E + (Is > 0 ? 1 : 0);  // <= 1025 groups: threads take g and g + 1024
+  int n[2] = {0, 0}, c13[2] = {0, 0}, c2[2] = {0, 0};
+  for (int q = 0; q < 2; ++q) {
+    const int g = threadIdx.x + q * 1024;
+    if (g < G) {
+      n[q] = g < E ? offsets[g + 1] - offsets[g] : T;
+      const int tt = (n[q] + BN - 1) / BN;
+      c13[q] = tt * ((g < E ? I : Is) / 64);
+      c2[q] = tt * (H / 128);
     }
-    base13[G] = a;
-    base2[G] = b;
-    *n13 = a;
-    *n2 = b;
   }
-  __syncthreads();
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    const int n = ntok(g);
-    const int tt = (n + BN - 1) / BN;
+  // second group of a thread (only the shared expert when E == 1024) follows all first groups
+  const int b13 = block_excl_scan_1024(c13[0], wt13, &tot13);
+  const int b2 = block_excl_scan_1024(c2[0], wt2, &tot2);
+  int base13[2] = {b13, tot13}, base2[2] = {b2, tot2};
+  if (threadIdx.x == 0) {
+    *n13 = tot13 + c13[1];
+    *n2 = tot2 + c2[1];
+  }
+  for (int q = 0; q < 2; ++q) {
+    const int g = threadIdx.x + q * 1024;
+    if (g >= G || (q == 1 && threadIdx.x != 0)) continue;
+    const int tt = (n[q] + BN - 1) / BN;
     const int nb13 = (g < E ? I : Is) / 64, nb2 = H / 128;
     for (int i = 0; i < tt; ++i) {
-      const int n0 = i * BN, nn = min(BN, n - n0);
-      for (int bb = 0; bb < nb13; ++bb) t13[base13[g] + i * nb13 + bb] = TcTile{g, bb * 64, n0, nn};
-      for (int bb = 0; bb < nb2; ++bb) t2[base2[g] + i * nb2 + bb] = TcTile{g, bb * 128, n0, nn};
+      const int n0 = i * BN, nn = min(BN, n[q] - n0);
+      for (int bb = 0; bb < nb13; ++bb) t13[base13[q] + i * nb13 + bb] = TcTile{g, bb * 64, n0, nn};
+      for (int bb = 0; bb < nb2; ++bb) t2[base2[q] + i * nb2 + bb] = TcTile{g, bb * 128, n0, nn};
     }
   }
 }
@@ -632,6 +690,10 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   P.ys = a.ys;
 
   P.mode = kW13;
+  P.w_codes = a.w.w13_codes;
+  P.sh_codes = reinterpret_cast<const uint8_t*>(a.w.sh_w13);
+  P.b_routed = xperm;
+  P.b_shared = x16;
   P.tiles = t13;
   P.ntiles = counts;
   P.w_scales = a.w.w13_scales;
@@ -641,6 +703,10 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   if (e != cudaSuccess) return e;
 
   P.mode = kW2;
+  P.w_codes = a.w.w2_codes;
+  P.sh_codes = reinterpret_cast<const uint8_t*>(a.w.sh_w2);
+  P.b_routed = reinterpret_cast<const __half*>(a.h);
+  P.b_shared = reinterpret_cast<const __half*>(a.hs);
   P.tiles = t2;
   P.ntiles = counts + 1;
   P.w_scales = a.w.w2_scales;

@@ -4,163 +4,123 @@
 // norm_topk_prob, routed_scaling_factor; hash layers per "DeepSeek-V4-Flash
 // export design", section "Source configuration").
 //
-// Learned routing, two kernels:
-//  * k_route_scores: gate GEMV s[t, e] = sqrt(softplus(x[t] . gate[e])). One
-//    CTA covers 32 experts x 8 tokens; each warp owns 4 experts and walks H in
-//    16-byte pieces (8 bf16), with the 8 token rows staged in shared memory.
-//    bf16 products are exact in fp32; accumulation is fp32.
-//  * k_route_select: one warp per token; k rounds of a warp arg-max over
-//    s + bias (value descending, expert id ascending on ties), ids emitted in
-//    ascending order, weights = scale * s[id] / sum s[ids] from the unbiased
-//    scores.
-// Hash routing, one kernel (k_route_hash): one warp per token reads its
-// tid2eid row and computes only the k needed gate dot products.
+//  * k_route_mma: per CTA 32 tokens x all experts; the gate
+//    GEMV runs as a bf16 tensor-core GEMM (exact products, fp32 sums), and
+//    sqrt(softplus), the biased top-k (ties to the lower id, ids ascending)
+//    and the weights (unbiased scores, normalised, x routed_scaling_factor)
+//    follow from shared memory in the same kernel.
+//    Hash routing (first layers) uses the same kernel: the scores at the
+//    tid2eid row's experts give the weights.
+// The decode-sized fused variant is in decode_prep.cu.
 #include "launch.cuh"
+#include "ptx.cuh"
 #include "route_dev.cuh"
 #include "v4moe_internal.cuh"
 
 namespace v4moe {
 namespace {
 
-constexpr int kScoreTokens = 8;    // tokens per CTA
-constexpr int kScoreExperts = 32;  // experts per CTA (4 per warp)
-constexpr int kSelectWarps = 8;
 
-__device__ __forceinline__ void fma_bf16x8(float& acc, const uint4& g, const uint4& x) {
-  acc = fmaf(bf16_lo(g.x), bf16_lo(x.x), acc);
-  acc = fmaf(bf16_hi(g.x), bf16_hi(x.x), acc);
-  acc = fmaf(bf16_lo(g.y), bf16_lo(x.y), acc);
-  acc = fmaf(bf16_hi(g.y), bf16_hi(x.y), acc);
-  acc = fmaf(bf16_lo(g.z), bf16_lo(x.z), acc);
-  acc = fmaf(bf16_hi(g.z), bf16_hi(x.z), acc);
-  acc = fmaf(bf16_lo(g.w), bf16_lo(x.w), acc);
-  acc = fmaf(bf16_hi(g.w), bf16_hi(x.w), acc);
-}
+// Learned routing on tensor cores: per CTA 32 tokens x all experts,
+// logits = x . gate^T with bf16 mma.sync (exact products, fp32 sums), then
+// sqrt(softplus) and the biased top-k selection from shared memory.
+// K is walked in 64-element slices, double-buffered with cp.async; rows are
+// stored with their 16-byte chunks XOR-swizzled by (row & 7) so that the
+// ldmatrix reads are conflict-free.
+constexpr int kRmTok = 32;     // tokens per CTA
+constexpr int kRmExp = 256;    // experts per pass (8 warps x 32)
+constexpr int kRmBK = 64;
 
-__device__ __forceinline__ float warp_sum(float v) {
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return uint32_t(row * 128 + ((chunk ^ (row & 7)) << 4)); }
+
+template <bool HASH>
+__global__ void __launch_bounds__(256) k_route_mma(int T, int H, int E, int k, int vocab, float routed_scale,
+                                                   const __nv_bfloat16* __restrict__ x,
+                                                   const __nv_bfloat16* __restrict__ gate,
+                                                   const float* __restrict__ bias,
+                                                   const int32_t* __restrict__ token_ids,
+                                                   const int32_t* __restrict__ tid2eid,
+                                                   int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+                                                   uint32_t* status) {
+  extern __shared__ __align__(128) char sm[];
+  char* As = sm;                                   // [2][32 rows][128 B]
+  char* Bs = sm + 2 * kRmTok * 128;                // [2][256 rows][128 B]
+  float* sc = reinterpret_cast<float*>(Bs + 2 * kRmExp * 128);  // [32][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * kRmTok;
+  const int nk = H / kRmBK;
+  for (int e0 = 0; e0 < E; e0 += kRmExp) {
+    auto load = [&](int kb, int buf) {
+      char* a = As + buf * kRmTok * 128;
+      char* b = Bs + buf * kRmExp * 128;
+      {  // x: 32 rows x 8 chunks, one per thread
+        const int row = threadIdx.x >> 3, ch = threadIdx.x & 7;
+        const bool ok = t0 + row < T;
+        cp_async16_zfill(a + swz(row, ch), x + size_t(ok ? t0 + row : 0) * H + kb * kRmBK + ch * 8, ok);
+      }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-__global__ void __launch_bounds__(256) k_route_scores(int T, int H, int E,
-                                                      const __nv_bfloat16* __restrict__ x,
-                                                      const __nv_bfloat16* __restrict__ gate,
-                                                      float* __restrict__ scores) {
-  extern __shared__ __align__(16) uint4 xs[];  // [kScoreTokens][H/8]
-  const int t0 = blockIdx.y * kScoreTokens;
-  const int e0 = blockIdx.x * kScoreExperts;
-  const int pieces = H / 8;
-  for (int i = threadIdx.x; i < kScoreTokens * pieces; i += blockDim.x) {
-    const int t = i / pieces, p = i % pieces;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (t0 + t < T) v = reinterpret_cast<const uint4*>(x + size_t(t0 + t) * H)[p];
-    xs[i] = v;
+      for (int i = 0; i < 8; ++i) {  // gate: 256 rows x 8 chunks
+        const int idx = threadIdx.x + i * 256;
+        const int row = idx >> 3, ch = idx & 7;
+        const bool ok = e0 + row < E;
+        cp_async16_zfill(b + swz(row, ch), gate + size_t(ok ? e0 + row : 0) * H + kb * kRmBK + ch * 8, ok);
+      }
+      cp_async_commit();
+    };
+    float acc[2][4][4] = {};
+    load(0, 0);
+    for (int kb = 0; kb < nk; ++kb) {
+      if (kb + 1 < nk) {
+        load(kb + 1, (kb + 1) & 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      const uint32_t a = smem_u32(As + (kb & 1) * kRmTok * 128);
+      const uint32_t b = smem_u32(Bs + (kb & 1) * kRmExp * 128);
+#pragma unroll
+      for (int kk = 0; kk < kRmBK / 16; ++kk) {
+        uint32_t af[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          ldmatrix_x4(af[mt][0], af[mt][1], af[mt][2], af[mt][3], a + swz(row, kk * 2 + (lane >> 4)));
+        }
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {  // pairs of n8 tiles
+          const int row = warp * 32 + np * 16 + (lane & 7) + (lane >> 4) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4(b0, b1, b2, b3, b + swz(row, kk * 2 + ((lane >> 3) & 1)));
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt) {
+            mma_16816_bf16(acc[mt][2 * np], af[mt], b0, b1);
+            mma_16816_bf16(acc[mt][2 * np + 1], af[mt], b2, b3);
+          }
+        }
+      }
+      __syncthreads();
+    }
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tok = mt * 16 + g + (i >> 1) * 8;
+          const int e = e0 + warp * 32 + nt * 8 + 2 * t + (i & 1);
+          if (e < E) sc[tok * E + e] = sqrt_softplus_f(acc[mt][nt][i]);
+        }
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float acc[4][kScoreTokens];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int t = 0; t < kScoreTokens; ++t) acc[a][t] = 0.0f;
-  const uint4* grow[4];
-  bool live[4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int e = e0 + warp * 4 + a;
-    live[a] = e < E;
-    grow[a] = reinterpret_cast<const uint4*>(gate + size_t(live[a] ? e : 0) * H);
-  }
-  for (int p = lane; p < pieces; p += 32) {
-    uint4 g[4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) g[a] = __ldg(grow[a] + p);
-#pragma unroll
-    for (int t = 0; t < kScoreTokens; ++t) {
-      const uint4 xv = xs[t * pieces + p];
-#pragma unroll
-      for (int a = 0; a < 4; ++a) fma_bf16x8(acc[a][t], g[a], xv);
-    }
-  }
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int t = 0; t < kScoreTokens; ++t) acc[a][t] = warp_sum(acc[a][t]);
-  if (lane == 0) {
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      if (!live[a]) continue;
-      const int e = e0 + warp * 4 + a;
-#pragma unroll
-      for (int t = 0; t < kScoreTokens; ++t)
-        if (t0 + t < T) scores[size_t(t0 + t) * E + e] = sqrt_softplus_f(acc[a][t]);
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kSelectWarps * 32) k_route_select(
-    int T, int E, int k, float routed_scale, const float* scores, const float* __restrict__ bias,
-    int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
-  const int warp = threadIdx.x >> 5;
-  const int t = blockIdx.x * kSelectWarps + warp;
-  if (t >= T) return;
-  select_learned_warp(t, E, k, routed_scale, scores + size_t(t) * E, bias, topk_ids, topk_w);
-}
-
-__global__ void __launch_bounds__(kSelectWarps * 32) k_route_hash(
-    int T, int H, int E, int k, int vocab, float routed_scale, const __nv_bfloat16* __restrict__ x,
-    const __nv_bfloat16* __restrict__ gate, const int32_t* __restrict__ token_ids,
-    const int32_t* __restrict__ tid2eid, int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
-    uint32_t* status) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kSelectWarps + warp;
-  if (t >= T) return;
-  const int tok = token_ids[t];
-  const bool tok_ok = tok >= 0 && tok < vocab;
-  int id[8];
-  bool ok[8];
-  bool any_bad = !tok_ok;
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    id[r] = 0;
-    ok[r] = false;
-    if (r < k && tok_ok) {
-      const int e = tid2eid[size_t(tok) * k + r];
-      ok[r] = e >= 0 && e < E;
-      id[r] = ok[r] ? e : 0;
-      any_bad |= !ok[r];
-    }
-  }
-  if (any_bad && lane == 0) atomicOr(status, tok_ok ? kStatusBadExpertId : kStatusBadTokenId);
-  const uint4* xr = reinterpret_cast<const uint4*>(x + size_t(t) * H);
-  float acc[8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) acc[r] = 0.0f;
-  for (int p = lane; p < H / 8; p += 32) {
-    const uint4 xv = __ldg(xr + p);
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r < k) fma_bf16x8(acc[r], __ldg(reinterpret_cast<const uint4*>(gate + size_t(id[r]) * H) + p), xv);
-  }
-  float sv[8];
-  float sum = 0.0f;
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    sv[r] = (r < k && ok[r]) ? sqrt_softplus_f(warp_sum(acc[r])) : 0.0f;
-    sum += sv[r];
-  }
-  if (lane < k) {
-    float myv = 0.0f;
-    int myid = 0;
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r == lane) {
-        myv = sv[r];
-        myid = id[r];
-      }
-    topk_ids[size_t(t) * k + lane] = myid;
-    topk_w[size_t(t) * k + lane] = sum > 0.0f ? routed_scale * (myv / sum) : 0.0f;
+  for (int tt = warp; tt < kRmTok; tt += 8) {
+    if (t0 + tt >= T) continue;
+    if (HASH)
+      select_hash_warp<true>(t0 + tt, E, k, vocab, routed_scale, sc + tt * E, token_ids, tid2eid, topk_ids, topk_w,
+                             status);
+    else
+      select_learned<false>(t0 + tt, E, k, routed_scale, sc + tt * E, bias, topk_ids, topk_w);
   }
 }
 
@@ -170,22 +130,19 @@ cudaError_t launch_route(const v4moe_config& c, int T, const __nv_bfloat16* x,
                          const __nv_bfloat16* gate, const float* bias, const int32_t* token_ids,
                          const int32_t* tid2eid, int32_t* topk_ids, float* topk_w, float* scores,
                          uint32_t* status, cudaStream_t st) {
+  (void)scores;
   if (T == 0) return cudaSuccess;
+  const size_t smem = size_t(2) * (kRmTok + kRmExp) * 128 + size_t(kRmTok) * c.n_experts * 4;
+  const dim3 grid((T + kRmTok - 1) / kRmTok);
   if (token_ids) {
-    const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
-    return launch_kernel("route_hash", k_route_hash, dim3(blocks), dim3(kSelectWarps * 32), 0, st, false,
-                         T, c.hidden, c.n_experts, c.top_k, c.vocab, c.routed_scale, x, gate, token_ids,
-                         tid2eid, topk_ids, topk_w, status);
+    set_smem(k_route_mma<true>, smem);
+    return launch_kernel("route_mma_hash", k_route_mma<true>, grid, dim3(256), smem, st, false, T, c.hidden,
+                         c.n_experts, c.top_k, c.vocab, c.routed_scale, x, gate, bias, token_ids, tid2eid, topk_ids,
+                         topk_w, status);
   }
-  const size_t smem = size_t(kScoreTokens) * c.hidden * 2;
-  set_smem(k_route_scores, smem);
-  dim3 grid((c.n_experts + kScoreExperts - 1) / kScoreExperts, (T + kScoreTokens - 1) / kScoreTokens);
-  cudaError_t e = launch_kernel("route_scores", k_route_scores, grid, dim3(256), smem, st, false, T, c.hidden,
-                                c.n_experts, x, gate, scores);
-  if (e != cudaSuccess) return e;
-  const int blocks = (T + kSelectWarps - 1) / kSelectWarps;
-  return launch_kernel("route_select", k_route_select, dim3(blocks), dim3(kSelectWarps * 32), 0, st, false, T,
-                       c.n_experts, c.top_k, c.routed_scale, (const float*)scores, bias, topk_ids, topk_w);
+  set_smem(k_route_mma<false>, smem);
+  return launch_kernel("route_mma", k_route_mma<false>, grid, dim3(256), smem, st, false, T, c.hidden, c.n_experts,
+                       c.top_k, c.vocab, c.routed_scale, x, gate, bias, token_ids, tid2eid, topk_ids, topk_w, status);
 }
 
 }  // namespace v4moe

@@ -1,6 +1,6 @@
 // Device-side routing and permutation building blocks shared by the router
 // kernels and the fused decode preparation kernel.
-//  * select_*_warp: one warp selects one token's experts and weights
+//  * select_learned / select_hash_warp: one warp selects one token's experts and weights
 //    ("Checked in its code" rows "Mixture of experts" and "Auxiliary-loss-free
 //    load balancing": top-k of s + bias, weights from the unbiased s, then
 //    normalised and multiplied by routed_scaling_factor).
@@ -13,90 +13,102 @@
 
 namespace v4moe {
 
-// Insertion sort of k <= 8 ids held identically by every lane.
-__device__ __forceinline__ void sort_ids8(int* id, int k) {
-  for (int i = 1; i < 8; ++i) {
-    if (i >= k) break;
-    const int v = id[i];
-    int j = i - 1;
-    while (j >= 0 && id[j] > v) {
-      id[j + 1] = id[j];
-      --j;
-    }
-    id[j + 1] = v;
+// Compare-exchange of (id, value) pairs held identically by every lane.
+__device__ __forceinline__ void cswap_pair(int& ia, float& va, int& ib, float& vb) {
+  if (ia > ib) {
+    const int ti = ia;
+    ia = ib;
+    ib = ti;
+    const float tv = va;
+    va = vb;
+    vb = tv;
   }
 }
 
-// Learned routing of token t given its E scores s (fp32): k rounds of a warp
-// arg-max over s + bias (largest value, then lowest id), ids written in
-// ascending order, w = scale * s[id] / sum of the k selected s.
-__device__ __forceinline__ void select_learned_warp(int t, int E, int k, float routed_scale,
-                                                    const float* s,
-                                                    const float* __restrict__ bias,
-                                                    int32_t* __restrict__ topk_ids,
-                                                    float* __restrict__ topk_w) {
+// Sort 8 (id, value) pairs by id (odd-even transposition with constant
+// indices, so the pairs stay in registers); unused entries carry INT_MAX.
+__device__ __forceinline__ void sort8_by_id(int id[8], float v[8]) {
+#pragma unroll
+  for (int pass = 0; pass < 8; ++pass) {
+#pragma unroll
+    for (int i = pass & 1; i + 1 < 8; i += 2) cswap_pair(id[i], v[i], id[i + 1], v[i + 1]);
+  }
+}
+
+// Learned routing of token t from its E scores s (fp32; SCORE_L2 reads them
+// through L2, for scores written by other CTAs of the same kernel): k rounds
+// of a warp arg-max over s + bias (largest value, then lowest id) that carry
+// the unbiased score along; ids written in ascending order; w = scale * s[id]
+// / sum of the selected s. Every load is issued before the first use.
+template <bool SCORE_L2>
+__device__ __forceinline__ void select_learned(int t, int E, int k, float routed_scale, const float* s,
+                                               const float* __restrict__ bias, int32_t* __restrict__ topk_ids,
+                                               float* __restrict__ topk_w) {
   const int lane = threadIdx.x & 31;
   const int nper = (E + 31) / 32;
-  float b[32];
+  float sv[32], b[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int e = lane + 32 * i;
-    float v = -INFINITY;
-    if (i < nper && e < E) {
-      v = __ldcg(s + e) + bias[e];
-      if (v != v) v = -INFINITY;  // NaN never wins
-    }
+    const int ec = (i < nper && e < E) ? e : 0;
+    sv[i] = SCORE_L2 ? __ldcg(s + ec) : s[ec];
+    b[i] = __ldg(bias + ec);
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int e = lane + 32 * i;
+    float v = sv[i] + b[i];
+    if (!(i < nper && e < E) || v != v) v = -INFINITY;  // NaN never wins
     b[i] = v;
   }
   uint32_t taken = 0;
   int id[8];
+  float sel[8];
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
-    if (r >= k) {
-      id[r] = 0x7fffffff;
-      continue;
-    }
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
+    id[r] = 0x7fffffff;
+    sel[r] = 0.0f;
+    if (r < k) {
+      float bv = -INFINITY, sb = 0.0f;
+      int be = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int e = lane + 32 * i;
-      if (i < nper && e < E && !((taken >> i) & 1u)) {
-        if (b[i] > bv || be == 0x7fffffff) {
+      for (int i = 0; i < 32; ++i) {
+        const int e = lane + 32 * i;
+        if (i < nper && e < E && !((taken >> i) & 1u) && (b[i] > bv || be == 0x7fffffff)) {
           bv = b[i];
           be = e;
+          sb = sv[i];
         }
       }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        const float os = __shfl_xor_sync(0xffffffffu, sb, o);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+          sb = os;
+        }
       }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      id[r] = be;
+      sel[r] = sb;
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    id[r] = be;
   }
-  sort_ids8(id, k);
+  sort8_by_id(id, sel);
   float sum = 0.0f;
-  float sv[8];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    sv[r] = (r < k) ? __ldcg(s + id[r]) : 0.0f;
-    sum += sv[r];
-  }
+  for (int r = 0; r < 8; ++r) sum += (r < k) ? sel[r] : 0.0f;
+  float myv = 0.0f;
+  int myid = 0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+    if (r == lane) {
+      myv = sel[r];
+      myid = id[r];
+    }
   if (lane < k) {
-    float myv = 0.0f;
-    int myid = 0;
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r == lane) {
-        myv = sv[r];
-        myid = id[r];
-      }
     topk_ids[size_t(t) * k + lane] = myid;
     topk_w[size_t(t) * k + lane] = routed_scale * (myv / sum);
   }
@@ -106,6 +118,7 @@ __device__ __forceinline__ void select_learned_warp(int t, int E, int k, float r
 // table", tid2eid): ids = tid2eid[token_id] in column order, weights from the
 // scores s at those ids. Out-of-range token ids / table entries flag the
 // status word and give expert 0 with weight 0.
+template <bool S_IN_SMEM = false>
 __device__ __forceinline__ void select_hash_warp(int t, int E, int k, int vocab, float routed_scale,
                                                  const float* s,
                                                  const int32_t* __restrict__ token_ids,
@@ -122,7 +135,7 @@ __device__ __forceinline__ void select_hash_warp(int t, int E, int k, int vocab,
     ok = e >= 0 && e < E;
     if (!ok) e = 0;
   }
-  const float v = ok ? __ldcg(s + e) : 0.0f;
+  const float v = ok ? (S_IN_SMEM ? s[e] : __ldcg(s + e)) : 0.0f;
   float sum = v;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
