@@ -1,32 +1,51 @@
-// Decode-sized expert path (at most 8 tokens, so at most 8 per expert):
-// weight-streaming grouped GEMV on warp-level tensor-core MMA.
+// Decode-sized batches (at most 8 tokens): the layer as three kernels chained
+// by programmatic dependent launch, streaming every weight byte once.
 //
-// What it computes ("Checked in its code" rows "SwiGLU feed-forward", "Shared
+// What it computes ("Checked in its code" rows "Mixture of experts",
+// "Auxiliary-loss-free load balancing", "SwiGLU feed-forward", "Shared
 // expert"; "config.json" experts_w4a16 / linears_w8a16):
-//   k_dec_w13: per group (routed expert or shared expert) and 8 output
-//              channels j: [g; u] = W13[{j, I+j}] x_t for the group's tokens,
-//              h_t[j] = silu(min(g, L)) * clamp(u, -L, L), stored as f16.
-//   k_dec_w2:  per 16 output rows m (owner computes): the shared expert, then
-//              every routed expert in ascending id: y = W2[m] h_t and
-//              out[t, m] += w[t, j] * y (weight 1 for the shared expert); the
-//              sum is written once as bf16. Fixed order, no output atomics in
-//              global memory.
+//   layer mode: s[t, e] = sqrt(softplus(gate[e] . x_t)), top-k of s + bias (or
+//   the token-id hash table), w = scale * s / sum; forward mode takes ids and
+//   weights from the caller. Then, for the shared expert and every routed
+//   expert the batch hits,
+//     h = silu(min(g, L)) * clamp(u, -L, L),   [g; u] = W13 x_t,
+//     out_t = W2_shared hs_t + sum over the token's experts of w * W2_e h.
 //
-// How:
-//  * Everything the CTA reads arrives by 1-D bulk async copies into shared
-//    memory, tracked by mbarriers with bounded waits: the weight tile (16 rows,
-//    one copy per row into a padded stride), its E8M0 scale rows, and the
-//    activation rows, which the preparation step stored as f16 in the MMA's
-//    K order (decode_logical_index) with a per-token power-of-two scale.
-//  * Weights become exact f16 MMA operands: E2M1 pairs via
-//    cvt.rn.f16x2.e2m1x2, int8 via an exact magic-number conversion. The E8M0
-//    group scale is applied to the operand as an exact power of two relative
-//    to the row's largest group exponent; the row factor multiplies the fp32
-//    result. Exact for every group within 36 binades of its row's largest.
-//  * mma.sync m16n8k16 with fp32 accumulation; the 8 warps split K and their
-//    partial tiles are summed in warp order through shared memory.
-//  * The shared expert's CTAs start streaming weights before the routing is
-//    known (programmatic dependent launch); routed CTAs wait for it.
+// Kernels:
+//  * k_dec_route: router scores (one warp per expert); the last CTA to finish
+//    selects each token's experts and publishes the batch's routing tables
+//    (distinct experts in ascending id, token masks, weights) and the
+//    permutation outputs. In forward mode one CTA publishes the tables of the
+//    caller's routing.
+//  * k_dec_w13: one CTA per SM, two groups of eight warps. Work items are w13
+//    slabs (8 channels of a routed expert: 8 gate rows and the 8 matching up
+//    rows; or 4 + 4 int8 rows of the shared expert), numbered shared first,
+//    then routed expert by expert; CTA b takes items b, b + G, ... as its ring
+//    positions 0, 1, .... Before the routing is known the CTA asks L2 for its
+//    shared slabs and for its share of the shared w2 rows; after it, for all
+//    of its routed slabs and its share of the routed w2 rows, so the HBM
+//    stream runs ahead of the shared-memory ring. Warp i of a group owns the
+//    128-wide K blocks i, i + 8, ... of a slab, multiplies them by the
+//    activations with mma.sync m16n8k16 (f16 operands, fp32 accumulation, the
+//    tokens as the 8 columns) and posts its partial tile to shared memory; the
+//    last warp to post sums the partials in warp order, refills the stage and
+//    writes h as f16 (routed: w * h).
+//  * k_dec_w2: one CTA per SM, sixteen warps owning K blocks i, i + 16, ....
+//    CTA b owns the 16-row output blocks b, b + G, ... and goes through the
+//    shared expert and every routed expert for each of them; a stage holds
+//    the expert's 16 weight rows and the intermediates of its tokens. The sum
+//    over experts (shared first, then ascending id) is formed in registers and
+//    written once as bf16, so the result does not depend on timing.
+//
+// Operands are exact: E2M1 pairs via cvt.rn.f16x2.e2m1x2, int8 via a
+// magic-number conversion; the E8M0 group scale multiplies the f16 operand as
+// a power of two relative to the largest exponent among the warp's groups of
+// that row, and the rest is applied in fp32. Activations are f16, scaled per
+// token by a power of two that puts the row maximum in [2^14, 2^15).
+//
+// No CTA waits on another CTA: data crosses kernels only at the programmatic
+// launch boundaries (griddepcontrol.wait), which also order memory. Every
+// mbarrier wait is bounded and flags the status word.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -39,25 +58,46 @@
 namespace v4moe {
 namespace {
 
-constexpr int kDW = 8;                 // warps per CTA
-constexpr int kDThreads = kDW * 32;
-constexpr int kTileRows = 16;          // weight rows per tile (one m16 MMA tile)
-constexpr int kMaxStages = 4;
-constexpr uint32_t kWaitTries = 1u << 20;
+constexpr int kGW = 8;             // warps per consumer group (w13 kernel)
+constexpr int kThreads = 16 * 32;  // both slab kernels
+constexpr int kStages13 = 5;
+constexpr int kMaxStages2 = 6;
+constexpr int kNJ = 4;             // K blocks per warp held in registers (K <= 4096)
+constexpr int kMaxHit = 64;        // distinct routed experts of a batch (T * k <= 64)
+constexpr uint32_t kBarTries = 1u << 20;
 
-enum { kMx = 0, kS8 = 1 };
+// Control block words (workspace): the ticket is zero at rest; the tables are
+// rewritten by every routing.
+enum Ctl : int {
+  cTicket = 0,
+  cEpoch = 16,        // calls so far; scores are tagged with epoch + 1
+  cNh = 32,
+  cHit = 64,          // [kMaxHit] expert id per list index
+  cMask = cHit + 64,  // [kMaxHit] bit per token routed to the expert
+  cW = cMask + 64,    // [kMaxHit][8] float weight per (expert, token)
+  cScores = 1024,     // [8][1024] u64: (tag << 32) | score bits, 8-byte aligned
+  cWords = cScores + 2 * 8 * 1024,
+};
 
 struct DecParams {
-  int T, H, I, Is, E, k;
-  float limit;
-  int n_shared_ctas;             // k_dec_w13: CTAs [0, n) do the shared expert
-  int stages;
+  int T, H, I, Is, E, k, vocab;
+  float limit, routed_scale;
+  int layer_mode;
   int stage_bytes;
-  const __half* xlog;            // [T, H] decode layout
-  const int* sigma;              // [T]
-  const int32_t* offsets;
-  const int32_t* sorted_slot;
-  const float* topk_w;
+  int nstages;  // w2 ring depth
+  int w2_per;   // 16-row output blocks per w2 CTA
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* gate;
+  const float* bias;
+  const int32_t* token_ids;
+  const int32_t* tid2eid;
+  int32_t* topk_ids;  // layer mode: written; forward mode: read
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_slot;
+  int32_t* slot_pos;
+  float* scores;  // [T, E]
   const uint8_t* w13_codes;
   const uint8_t* w13_scales;
   const uint8_t* w2_codes;
@@ -66,522 +106,925 @@ struct DecParams {
   const float* sh13_scale;
   const int8_t* sh2;
   const float* sh2_scale;
-  __half* hlog;                  // [T*k, I] routed intermediates (sorted order, decode layout)
-  __half* hslog;                 // [T, I_s] shared intermediates (decode layout)
-  __nv_bfloat16* out;
+  __half* dh;  // [kMaxHit, T, I] weighted routed intermediates
+  __half* hs;  // [T, Is] shared intermediates
+  uint32_t* ctl;
   uint32_t* status;
+  __nv_bfloat16* out;
 };
 
-__host__ __device__ inline int tile_stride(int fmt, int K) {
-  const int rb = fmt == kMx ? K / 2 : K;
-  return fmt == kMx ? rb + ((rb % 128 == 0) ? 64 : 0) : rb + 16;
-}
-__host__ __device__ inline int xs_stride(int K) { return K * 2 + 16; }
-// Stage: weight tile followed by the 16 scale rows (MX only).
-__host__ __device__ inline int stage_size(int fmt, int K) {
-  return kTileRows * tile_stride(fmt, K) + (fmt == kMx ? kTileRows * (K / 32) : 0);
-}
-
-__device__ __forceinline__ size_t umin_(size_t a, size_t b) { return a < b ? a : b; }
+// Routing tables as the slab kernels keep them in shared memory.
+struct Tables {
+  int nh;
+  int hit[kMaxHit];
+  uint32_t mask[kMaxHit];
+  float w[kMaxHit * 8];
+};
 
 __device__ __forceinline__ float pow2f(int e) {
   e = max(-126, min(127, e));
   return __int_as_float((e + 127) << 23);
 }
 
-// Bounded wait that flags a timeout in the status word.
-__device__ __forceinline__ bool wait_or_flag(uint64_t* bar, uint32_t parity, uint32_t* status) {
-  if (mbar_wait_bounded(bar, parity, kWaitTries)) return true;
-  atomicOr(status, kStatusTimeout);
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const DecParams& P) {
+  if (mbar_wait_bounded(bar, parity, kBarTries)) return true;
+  atomicOr(P.status, kStatusTimeout);
   return false;
 }
 
-// Issue the copies of one weight tile (+ scale rows) into a stage; thread 0.
-// rows[i] is the global row of tile row i; rows 0-7 and 8-15 are each
-// contiguous, so their scale rows come in two copies.
-__device__ __forceinline__ void issue_tile(char* stage, int fmt, int K, const uint8_t* base,
-                                           const uint8_t* scales, const int* rows, uint64_t* bar) {
-  const int rb = fmt == kMx ? K / 2 : K;
-  const int ws = tile_stride(fmt, K);
-  const int G = K / 32;
-  const uint32_t bytes = uint32_t(kTileRows * rb + (fmt == kMx ? kTileRows * G : 0));
-  mbar_arrive_expect_tx(bar, bytes);
-#pragma unroll 1
-  for (int i = 0; i < kTileRows; ++i) bulk_g2s(stage + i * ws, base + size_t(rows[i]) * rb, uint32_t(rb), bar);
-  if (fmt == kMx) {
-    char* sc = stage + kTileRows * ws;
-    bulk_g2s(sc, scales + size_t(rows[0]) * G, uint32_t(8 * G), bar);
-    bulk_g2s(sc + 8 * G, scales + size_t(rows[8]) * G, uint32_t(8 * G), bar);
-  }
+// 14 - floor(log2 m) for the largest bf16 magnitude bits m of a row (0 for an
+// all-zero row), clamped to [-120, 120]: 2^sigma * max lies in [2^14, 2^15).
+__device__ __forceinline__ int sigma_of(uint32_t mx) {
+  if (mx == 0) return 0;
+  const int ef = int(mx >> 7);
+  const int sg = ef == 0 ? 120 : 141 - ef;
+  return max(-120, min(120, sg));
 }
 
-// Largest E8M0 exponent of each of the 16 scale rows in shared memory.
-__device__ __forceinline__ void row_max_exp(const uint8_t* sc, int G, int* rowx) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int r = warp; r < kTileRows; r += kDW) {
-    int m = 0;
-    for (int g = lane; g < G; g += 32) m = max(m, int(sc[r * G + g]));
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t w) {
+  return max(m, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
+}
+
+// Whole CTA; the caller synchronises afterwards.
+__device__ __forceinline__ void read_tables(Tables& tb, const DecParams& P) {
+  const int nh = int(P.ctl[cNh]);
+  for (int i = threadIdx.x; i < nh; i += blockDim.x) {
+    tb.hit[i] = int(P.ctl[cHit + i]);
+    tb.mask[i] = P.ctl[cMask + i];
+  }
+  for (int i = threadIdx.x; i < nh * 8; i += blockDim.x) tb.w[i] = reinterpret_cast<const float*>(P.ctl + cW)[i];
+  if (threadIdx.x == 0) tb.nh = nh;
+}
+
+// ---------------------------------------------------------------- slab products
+
+// MXFP4 m16 tile: rows g and g + 8 of the tile at ra / rb (codes of 128-wide
+// K block kb at kb * 64), their E8M0 scale rows at sa / sb. The warp's K
+// blocks kb = wi + KS j (j < NJ, kb < nkb) multiply B[j]. Even and odd MMA
+// steps go to separate accumulators; fa / fb get the fp32 factors of the two
+// rows.
+template <int NJ, int KS>
+__device__ __forceinline__ void tile_mx(const char* ra, const char* rb, const uint8_t* sa, const uint8_t* sb, int wi,
+                                        int nkb, const uint32_t (&B)[NJ][16], float (&ae)[4], float (&ao)[4],
+                                        float& fa, float& fb) {
+  const int t = threadIdx.x & 3;
+  int xa = 0, xb = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) rowx[r] = m;
+  for (int j = 0; j < NJ; ++j) {
+    const int kb = wi + KS * j;
+    if (kb < nkb) {
+      xa = max(xa, int(sa[4 * kb + t]));
+      xb = max(xb, int(sb[4 * kb + t]));
+    }
   }
-}
-
-// One warp's share (K blocks warp, warp + 8, ...) of a 16-row tile times the
-// staged activation rows (one n8 tile). acc: fp32 C fragment (rows g, g+8;
-// token columns 2t, 2t+1).
-template <int FMT>
-__device__ __forceinline__ void warp_tile_mma(const char* wt, int wstride, const uint8_t* sc, const char* xs,
-                                              int K, int nrows, const int* rowx, float acc[4]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int G = K / 32;
-  const int nblk = K / 128;
-  int tok = min(lane & 7, nrows - 1);
-  const uint32_t xaddr = smem_u32(xs + size_t(tok) * xs_stride(K)) + ((lane >> 3) & 1) * 16 + (lane >> 4) * 32;
-  const int xa = FMT == kMx ? rowx[g] : 0;
-  const int xb = FMT == kMx ? rowx[g + 8] : 0;
-  for (int b = warp; b < nblk; b += kDW) {
-    uint32_t A[8][4];
-    if (FMT == kMx) {
-      const uint4 qa = *reinterpret_cast<const uint4*>(wt + g * wstride + b * 64 + 16 * t);
-      const uint4 qb = *reinterpret_cast<const uint4*>(wt + (g + 8) * wstride + b * 64 + 16 * t);
-      const uint32_t sa = f16_pow2_bits(int(sc[g * G + 4 * b + t]) - xa + 13) * 0x10001u;
-      const uint32_t sb = f16_pow2_bits(int(sc[(g + 8) * G + 4 * b + t]) - xb + 13) * 0x10001u;
+  xa = max(xa, __shfl_xor_sync(0xffffffffu, xa, 1));
+  xa = max(xa, __shfl_xor_sync(0xffffffffu, xa, 2));
+  xb = max(xb, __shfl_xor_sync(0xffffffffu, xb, 1));
+  xb = max(xb, __shfl_xor_sync(0xffffffffu, xb, 2));
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int kb = wi + KS * j;
+    if (kb < nkb) {
+      const uint4 qa = *reinterpret_cast<const uint4*>(ra + kb * 64 + 16 * t);
+      const uint4 qb = *reinterpret_cast<const uint4*>(rb + kb * 64 + 16 * t);
+      const uint32_t fsa = f16_pow2_bits(int(sa[4 * kb + t]) - xa + 13) * 0x10001u;
+      const uint32_t fsb = f16_pow2_bits(int(sb[4 * kb + t]) - xb + 13) * 0x10001u;
       const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
       const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-      for (int wi = 0; wi < 4; ++wi) {
-        uint32_t fa[4], fb[4];
-        e2m1x8_to_f16x2(wa[wi], fa);
-        e2m1x8_to_f16x2(wb[wi], fb);
-        A[2 * wi][0] = hmul2_u32(fa[0], sa);
-        A[2 * wi][1] = hmul2_u32(fb[0], sb);
-        A[2 * wi][2] = hmul2_u32(fa[1], sa);
-        A[2 * wi][3] = hmul2_u32(fb[1], sb);
-        A[2 * wi + 1][0] = hmul2_u32(fa[2], sa);
-        A[2 * wi + 1][1] = hmul2_u32(fb[2], sb);
-        A[2 * wi + 1][2] = hmul2_u32(fa[3], sa);
-        A[2 * wi + 1][3] = hmul2_u32(fb[3], sb);
+      for (int u = 0; u < 4; ++u) {
+        uint32_t ca[4], cb[4];
+        e2m1x8_to_f16x2(wa[u], ca);
+        e2m1x8_to_f16x2(wb[u], cb);
+        const uint32_t A0[4] = {hmul2_u32(ca[0], fsa), hmul2_u32(cb[0], fsb), hmul2_u32(ca[1], fsa),
+                                hmul2_u32(cb[1], fsb)};
+        const uint32_t A1[4] = {hmul2_u32(ca[2], fsa), hmul2_u32(cb[2], fsb), hmul2_u32(ca[3], fsa),
+                                hmul2_u32(cb[3], fsb)};
+        mma_16816_f16(ae, A0, B[j][4 * u], B[j][4 * u + 1]);
+        mma_16816_f16(ao, A1, B[j][4 * u + 2], B[j][4 * u + 3]);
       }
-    } else {
-      const uint4* pa = reinterpret_cast<const uint4*>(wt + g * wstride + b * 128 + 32 * t);
-      const uint4* pb = reinterpret_cast<const uint4*>(wt + (g + 8) * wstride + b * 128 + 32 * t);
-      const uint4 qa0 = pa[0], qa1 = pa[1], qb0 = pb[0], qb1 = pb[1];
+    }
+  }
+  fa = pow2f(xa - 127 - 13);
+  fb = pow2f(xb - 127 - 13);
+}
+
+// int8 m16 tile: rows g and g + 8 at ra / rb (K block kb at (kb - kb0) * 128),
+// zero rows where `valid` is false. The warp's K blocks kb = wi + KS j inside
+// [kb0, kb1) multiply B[j].
+template <int NJ, int KS>
+__device__ __forceinline__ void tile_s8(const char* ra, const char* rb, bool valid, int kb0, int kb1, int wi,
+                                        const uint32_t (&B)[NJ][16], float (&ae)[4], float (&ao)[4]) {
+  const int t = threadIdx.x & 3;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int kb = wi + KS * j;
+    if (kb >= kb0 && kb < kb1) {
+      uint4 qa0 = make_uint4(0u, 0u, 0u, 0u), qa1 = qa0, qb0 = qa0, qb1 = qa0;
+      if (valid) {
+        const char* pa = ra + (kb - kb0) * 128 + 32 * t;
+        const char* pb = rb + (kb - kb0) * 128 + 32 * t;
+        qa0 = *reinterpret_cast<const uint4*>(pa);
+        qa1 = *reinterpret_cast<const uint4*>(pa + 16);
+        qb0 = *reinterpret_cast<const uint4*>(pb);
+        qb1 = *reinterpret_cast<const uint4*>(pb + 16);
+      }
       const uint32_t wa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
       const uint32_t wb[8] = {qb0.x, qb0.y, qb0.z, qb0.w, qb1.x, qb1.y, qb1.z, qb1.w};
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        s8x4_to_f16x2(wa[s], A[s][0], A[s][2]);
-        s8x4_to_f16x2(wb[s], A[s][1], A[s][3]);
+        uint32_t A[4];
+        s8x4_to_f16x2(wa[s], A[0], A[2]);
+        s8x4_to_f16x2(wb[s], A[1], A[3]);
+        if (s & 1)
+          mma_16816_f16(ao, A, B[j][2 * s], B[j][2 * s + 1]);
+        else
+          mma_16816_f16(ae, A, B[j][2 * s], B[j][2 * s + 1]);
       }
     }
-#pragma unroll
-    for (int sp = 0; sp < 4; ++sp) {
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4(b0, b1, b2, b3, xaddr + (b * 128 + sp * 32) * 2);
-      mma_16816_f16(acc, A[2 * sp], b0, b1);
-      mma_16816_f16(acc, A[2 * sp + 1], b2, b3);
-    }
   }
 }
 
-// Sum the 8 warps' C fragments in warp order; result valid in warp 0.
-__device__ __forceinline__ void reduce_warps(float acc[4], float* red) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) red[(warp * 4 + i) * 32 + lane] = acc[i];
-  __syncthreads();
-  if (warp == 0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float s = 0.f;
-      for (int w = 0; w < kDW; ++w) s += red[(w * 4 + i) * 32 + lane];
-      acc[i] = s;
-    }
-  }
-}
+// ---------------------------------------------------------------- routing kernel
 
-// Compact list of non-empty routed experts in ascending id (one warp).
-__device__ __forceinline__ int build_hit_list(const int32_t* offsets, int E, int* list) {
-  const int lane = threadIdx.x & 31;
-  int n = 0;
-  for (int base = 0; base < E; base += 32) {
-    const int e = base + lane;
-    const bool hit = e < E && offsets[e + 1] > offsets[e];
-    const unsigned m = __ballot_sync(0xffffffffu, hit);
-    if (hit) list[n + __popc(m & ((1u << lane) - 1u))] = e;
-    n += __popc(m);
-  }
-  return n;
-}
-
-struct SmemDec {
-  uint64_t bars[kMaxStages];
-  uint64_t xbar;
-  int rowx[kMaxStages][kTileRows];
-  int rows[kMaxStages][kTileRows];
-  int nlist;
+struct RouteSmem {
+  int is_last;
+  uint32_t bits[32];
+  int rank_base[32];
+  int cnt[kMaxHit];
+  int cum[kMaxHit + 1];
+  int hit[kMaxHit];
+  uint32_t mask[kMaxHit];
+  float wtab[kMaxHit * 8];
+  int ids[64];
+  float wts[64];
+  int32_t sel_ids[64];  // the selection's output, before it goes to global memory
+  float sel_w[64];
 };
 
-// ------------------------------------------------------------------ w13
-
-__global__ void __launch_bounds__(kDThreads) k_dec_w13(DecParams P) {
-  extern __shared__ __align__(128) char smem[];
-  SmemDec& S = *reinterpret_cast<SmemDec*>(smem);
-  int* list = reinterpret_cast<int*>(smem + 1024);
-  float* red = reinterpret_cast<float*>(smem + 1024 + ((P.E + 1) * 4 + 127) / 128 * 128);
-  char* stages = reinterpret_cast<char*>(red + kDW * 4 * 32);
-  char* xs = stages + size_t(P.stages) * P.stage_bytes;
-  const int H = P.H, T = P.T;
-  const bool shared_cta = int(blockIdx.x) < P.n_shared_ctas;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int fmt = shared_cta ? kS8 : kMx;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < P.stages; ++s) mbar_init(&S.bars[s], 1);
-    mbar_init(&S.xbar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  // ---- work range ----
-  int n_routed = 0, it0 = 0, it1 = 0, blk = 0;
-  if (shared_cta) {
-    blk = P.Is / 8;
-    const int per = (blk + P.n_shared_ctas - 1) / P.n_shared_ctas;
-    it0 = blockIdx.x * per;
-    it1 = min(blk, it0 + per);
-  } else {
-    pdl_wait();  // routing comes from the preparation kernel
-    if (warp == 0) {
-      const int n = build_hit_list(P.offsets, P.E, list);
-      if (lane == 0) S.nlist = n;
-    }
-    __syncthreads();
-    n_routed = S.nlist;
-    blk = P.I / 8;
-    const int n_items = n_routed * blk;
-    const int ctas = gridDim.x - P.n_shared_ctas;
-    const int per = (n_items + ctas - 1) / ctas;
-    it0 = (blockIdx.x - P.n_shared_ctas) * per;
-    it1 = min(n_items, it0 + per);
-  }
-  const int Ig = shared_cta ? P.Is : P.I;
-  auto item_group = [&](int it) { return shared_cta ? P.E : list[it / blk]; };
-  auto issue = [&](int it, int s) {  // thread 0
-    const int grp = item_group(it);
-    const int j0 = (it % blk) * 8;
-    for (int i = 0; i < kTileRows; ++i) S.rows[s][i] = i < 8 ? j0 + i : Ig + j0 + (i - 8);
-    const uint8_t* base = shared_cta ? reinterpret_cast<const uint8_t*>(P.sh13)
-                                     : P.w13_codes + size_t(grp) * 2 * P.I * (H / 2);
-    const uint8_t* scl = shared_cta ? nullptr : P.w13_scales + size_t(grp) * 2 * P.I * (H / 32);
-    issue_tile(stages + size_t(s) * P.stage_bytes, fmt, H, base, scl, S.rows[s], &S.bars[s]);
-  };
-  if (it0 < it1 && threadIdx.x == 0)
-    for (int s = 0; s < P.stages && it0 + s < it1; ++s) issue(it0 + s, s);
-  // Ask for every later tile of this CTA now, into L2: the whole weight stream
-  // of the kernel is then in flight at once and the ring's copies hit L2.
-  if (warp == 1) {
-    for (int it = it0 + P.stages + lane; it < it1; it += 32) {
-      const int grp = item_group(it);
-      const int j0 = (it % blk) * 8;
-      if (shared_cta) {
-        const uint8_t* b = reinterpret_cast<const uint8_t*>(P.sh13);
-        prefetch_l2_bulk(b + size_t(j0) * H, uint32_t(8 * H));
-        prefetch_l2_bulk(b + size_t(Ig + j0) * H, uint32_t(8 * H));
-      } else {
-        const uint8_t* b = P.w13_codes + size_t(grp) * 2 * P.I * (H / 2);
-        const uint8_t* sc = P.w13_scales + size_t(grp) * 2 * P.I * (H / 32);
-        prefetch_l2_bulk(b + size_t(j0) * (H / 2), uint32_t(8 * (H / 2)));
-        prefetch_l2_bulk(b + size_t(Ig + j0) * (H / 2), uint32_t(8 * (H / 2)));
-        prefetch_l2_bulk(sc + size_t(j0) * (H / 32), uint32_t(8 * (H / 32)));
-        prefetch_l2_bulk(sc + size_t(Ig + j0) * (H / 32), uint32_t(8 * (H / 32)));
+// Publishes the batch's routed experts (ascending ids), per (expert, token)
+// weights and token masks from topk ids / weights (global or shared memory);
+// one warp. Out-of-range ids are skipped and flagged. Returns the expert
+// count.
+__device__ int build_route_meta(RouteSmem& S, const DecParams& P, const int32_t* tids, const float* tw) {
+  const int lane = threadIdx.x & 31;
+  const int Sn = P.T * P.k;
+  S.bits[lane] = 0u;
+  __syncwarp();
+  bool bad = false;
+  for (int s = lane; s < 64; s += 32) {
+    int e = -1;
+    float w = 0.f;
+    if (s < Sn) {
+      e = tids[s];
+      w = tw[s];
+      if (e < 0 || e >= P.E) {
+        bad = true;
+        e = -1;
       }
     }
+    S.ids[s] = e;
+    S.wts[s] = w;
+    if (e >= 0) atomicOr(&S.bits[e >> 5], 1u << (e & 31));
   }
-  // The down projection of the same experts streams next: start moving its
-  // weights into L2 while this kernel runs (the routed CTAs split the hit
-  // experts' W2 blocks; the shared CTAs split the shared expert's).
-  if (warp == 2 && lane == 0) {
-    const int nctas = shared_cta ? P.n_shared_ctas : int(gridDim.x) - P.n_shared_ctas;
-    const int me = shared_cta ? int(blockIdx.x) : int(blockIdx.x) - P.n_shared_ctas;
-    if (shared_cta) {
-      const size_t total = size_t(H) * P.Is;
-      const size_t per = (total / nctas + 15) / 16 * 16;
-      const size_t a = size_t(me) * per;
-      if (a < total) prefetch_l2_range(reinterpret_cast<const uint8_t*>(P.sh2) + a, umin_(per, total - a));
-    } else if (n_routed > 0) {
-      const size_t codes = size_t(H) * (P.I / 2), scl = size_t(H) * (P.I / 32);
-      const size_t per_e = codes + scl;
-      const size_t total = per_e * n_routed;
-      const size_t per = (total / nctas + 15) / 16 * 16;
-      size_t a = size_t(me) * per;
-      const size_t b = umin_(total, a + per);
-      while (a < b) {
-        const int li = int(a / per_e);
-        size_t off = a - size_t(li) * per_e;
-        const size_t n = umin_(b - a, per_e - off);
-        const int e = list[li];
-        if (off < codes) {
-          const size_t nc = umin_(n, codes - off);
-          prefetch_l2_range(P.w2_codes + size_t(e) * codes + off, nc);
-          if (n > nc) prefetch_l2_range(P.w2_scales + size_t(e) * scl, n - nc);
-        } else {
-          prefetch_l2_range(P.w2_scales + size_t(e) * scl + (off - codes), n);
-        }
-        a += n;
-      }
-    }
-  }
-  if (shared_cta) pdl_wait();  // the activations come from the preparation kernel
-  if (it0 >= it1) return;
-
-  int staged = -1;
-  uint32_t xphase = 0;
-  for (int it = it0; it < it1; ++it) {
-    const int i = it - it0;
-    const int s = i % P.stages;
-    const uint32_t parity = uint32_t(i / P.stages) & 1u;
-    const int grp = item_group(it);
-    const int j0 = (it % blk) * 8;
-    const int r0 = shared_cta ? 0 : P.offsets[grp];
-    const int n = shared_cta ? T : P.offsets[grp + 1] - r0;
-    if (grp != staged) {
-      __syncthreads();  // readers of the previous activations are done
-      if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(&S.xbar, uint32_t(n * H * 2));
-        for (int r = 0; r < n; ++r) {
-          const int tok = shared_cta ? r : P.sorted_slot[r0 + r] / P.k;
-          bulk_g2s(xs + size_t(r) * xs_stride(H), P.xlog + size_t(tok) * H, uint32_t(H * 2), &S.xbar);
-        }
-      }
-      if (!wait_or_flag(&S.xbar, xphase, P.status)) break;
-      xphase ^= 1u;
-      staged = grp;
-    }
-    if (!wait_or_flag(&S.bars[s], parity, P.status)) break;
-    const char* st = stages + size_t(s) * P.stage_bytes;
-    const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + kTileRows * tile_stride(fmt, H));
-    if (fmt == kMx) row_max_exp(sc, H / 32, S.rowx[s]);
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (fmt == kMx)
-      warp_tile_mma<kMx>(st, tile_stride(kMx, H), sc, xs, H, n, S.rowx[s], acc);
-    else
-      warp_tile_mma<kS8>(st, tile_stride(kS8, H), nullptr, xs, H, n, S.rowx[s], acc);
-    reduce_warps(acc, red);
-    if (warp == 0) {
-      float fg, fu;
-      if (fmt == kMx) {
-        fg = pow2f(S.rowx[s][g] - 127 - 13);
-        fu = pow2f(S.rowx[s][g + 8] - 127 - 13);
-      } else {
-        fg = __ldg(P.sh13_scale + j0 + g);
-        fu = __ldg(P.sh13_scale + Ig + j0 + g);
-      }
-      __half* hout = shared_cta ? P.hslog : P.hlog;
-      const int L = decode_logical_index(j0 + g);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(P.status, kStatusBadExpertId);
+  __syncwarp();
+  const uint32_t word = S.bits[lane];
+  const int c = __popc(word);
+  int incl = c;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int nn = 2 * t + q;
-        if (nn < n) {
-          const int tok = shared_cta ? nn : P.sorted_slot[r0 + nn] / P.k;
-          const float inv = pow2f(-P.sigma[tok]);
-          const float gv = acc[q] * fg * inv;
-          const float uv = acc[2 + q] * fu * inv;
-          hout[size_t(r0 + nn) * Ig + L] = __float2half_rn(clamped_swiglu_f(gv, uv, P.limit));
-        }
-      }
-    }
-    __syncthreads();  // every warp is done with stage s
-    if (threadIdx.x == 0 && it + P.stages < it1) issue(it + P.stages, s);
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
   }
-  // Only reached early after a timeout: give the copies still in flight into
-  // this CTA's shared memory a bounded wait before leaving.
-  if (threadIdx.x == 0)
-    for (int s = 0; s < P.stages; ++s) mbar_wait_bounded(&S.bars[s], 0, 1);
+  S.rank_base[lane] = incl - c;
+  const int nh = __shfl_sync(0xffffffffu, incl, 31);
+  for (int i = lane; i < kMaxHit * 8; i += 32) S.wtab[i] = 0.f;
+  for (int i = lane; i < kMaxHit; i += 32) {
+    S.mask[i] = 0u;
+    S.cnt[i] = 0;
+  }
+  __syncwarp();
+  for (int s = lane; s < Sn; s += 32) {
+    const int e = S.ids[s];
+    if (e >= 0) {
+      const int r = S.rank_base[e >> 5] + __popc(S.bits[e >> 5] & ((1u << (e & 31)) - 1u));
+      const int tok = s / P.k;
+      S.hit[r] = e;
+      atomicAdd(&S.wtab[r * 8 + tok], S.wts[s]);
+      atomicOr(&S.mask[r], 1u << tok);
+      atomicAdd(&S.cnt[r], 1);
+    }
+  }
+  __syncwarp();
+  float* wg = reinterpret_cast<float*>(P.ctl + cW);
+  for (int i = lane; i < nh; i += 32) {
+    P.ctl[cHit + i] = uint32_t(S.hit[i]);
+    P.ctl[cMask + i] = S.mask[i];
+  }
+  for (int i = lane; i < nh * 8; i += 32) wg[i] = S.wtab[i];
+  if (lane == 0) P.ctl[cNh] = uint32_t(nh);
+  return nh;
 }
 
-// ------------------------------------------------------------------ w2 + combine
-
-__global__ void __launch_bounds__(kDThreads) k_dec_w2(DecParams P) {
-  extern __shared__ __align__(128) char smem[];
-  SmemDec& S = *reinterpret_cast<SmemDec*>(smem);
-  int* list = reinterpret_cast<int*>(smem + 1024);
-  float* red = reinterpret_cast<float*>(smem + 1024 + ((P.E + 2) * 4 + 127) / 128 * 128);
-  float* oacc = red + kDW * 4 * 32;                                   // [T][16]
-  char* stages = reinterpret_cast<char*>(oacc) + ((P.T * kTileRows * 4 + 127) / 128) * 128;
-  char* xs = stages + size_t(P.stages) * P.stage_bytes;
-  const int H = P.H, T = P.T;
-  const int m0 = blockIdx.x * kTileRows;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-
-  for (int i = threadIdx.x; i < T * kTileRows; i += kDThreads) oacc[i] = 0.f;
-  if (threadIdx.x < kTileRows)
-    for (int s = 0; s < kMaxStages; ++s) S.rows[s][threadIdx.x] = m0 + threadIdx.x;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < P.stages; ++s) mbar_init(&S.bars[s], 1);
-    mbar_init(&S.xbar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  const bool has_shared = P.Is > 0;
-  auto issue = [&](int gi, int s) {  // thread 0
-    const bool sh = gi == P.E;
-    const int Kg = sh ? P.Is : P.I;
-    const uint8_t* base = sh ? reinterpret_cast<const uint8_t*>(P.sh2) : P.w2_codes + size_t(gi) * H * (P.I / 2);
-    const uint8_t* scl = sh ? nullptr : P.w2_scales + size_t(gi) * H * (P.I / 32);
-    issue_tile(stages + size_t(s) * P.stage_bytes, sh ? kS8 : kMx, Kg, base, scl, S.rows[s], &S.bars[s]);
-  };
-  // The shared expert goes first; its weights do not depend on the routing.
-  if (threadIdx.x == 0 && has_shared) issue(P.E, 0);
-  pdl_wait();  // h and the routing come from the previous kernels
-  if (warp == 0) {
-    if (has_shared && lane == 0) list[0] = P.E;
-    const int n = build_hit_list(P.offsets, P.E, list + (has_shared ? 1 : 0));
-    if (lane == 0) S.nlist = n + (has_shared ? 1 : 0);
-  }
-  __syncthreads();
-  const int nl = S.nlist;
-  if (threadIdx.x == 0)
-    for (int s = has_shared ? 1 : 0; s < P.stages && s < nl; ++s) issue(list[s], s);
-
-  uint32_t xphase = 0;
-  bool ok = true;
-  for (int li = 0; li < nl && ok; ++li) {
-    const int s = li % P.stages;
-    const uint32_t parity = uint32_t(li / P.stages) & 1u;
-    const int gi = list[li];
-    const bool sh = gi == P.E;
-    const int fmt = sh ? kS8 : kMx;
-    const int Kg = sh ? P.Is : P.I;
-    const int r0 = sh ? 0 : P.offsets[gi];
-    const int n = sh ? T : P.offsets[gi + 1] - r0;
-    if (threadIdx.x == 0) {
-      const __half* src = sh ? P.hslog : P.hlog;
-      mbar_arrive_expect_tx(&S.xbar, uint32_t(n * Kg * 2));
-      for (int r = 0; r < n; ++r)
-        bulk_g2s(xs + size_t(r) * xs_stride(Kg), src + size_t(r0 + r) * Kg, uint32_t(Kg * 2), &S.xbar);
-    }
-    ok = wait_or_flag(&S.bars[s], parity, P.status);
-    ok = wait_or_flag(&S.xbar, xphase, P.status) && ok;
-    xphase ^= 1u;
-    if (!ok) break;
-    const char* st = stages + size_t(s) * P.stage_bytes;
-    const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + kTileRows * tile_stride(fmt, Kg));
-    if (fmt == kMx) row_max_exp(sc, Kg / 32, S.rowx[s]);
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    if (fmt == kMx)
-      warp_tile_mma<kMx>(st, tile_stride(kMx, Kg), sc, xs, Kg, n, S.rowx[s], acc);
-    else
-      warp_tile_mma<kS8>(st, tile_stride(kS8, Kg), nullptr, xs, Kg, n, S.rowx[s], acc);
-    reduce_warps(acc, red);
-    if (warp == 0) {
-      float fa, fb;
-      if (fmt == kMx) {
-        fa = pow2f(S.rowx[s][g] - 127 - 13);
-        fb = pow2f(S.rowx[s][g + 8] - 127 - 13);
-      } else {
-        fa = __ldg(P.sh2_scale + m0 + g);
-        fb = __ldg(P.sh2_scale + m0 + g + 8);
-      }
+// Stable counting sort of the batch's slots by expert (layer-mode outputs),
+// from the tables build_route_meta left in shared memory; one warp.
+__device__ void write_permutation(RouteSmem& S, const DecParams& P, int nh) {
+  const int lane = threadIdx.x & 31;
+  const int Sn = P.T * P.k;
+  const int c0 = 2 * lane < nh ? S.cnt[2 * lane] : 0;
+  const int c1 = 2 * lane + 1 < nh ? S.cnt[2 * lane + 1] : 0;
+  int incl = c0 + c1;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int nn = 2 * t + q;
-        if (nn < n) {
-          int tok;
-          float wgt;
-          if (sh) {
-            tok = nn;
-            wgt = 1.0f;
-          } else {
-            const int slot = P.sorted_slot[r0 + nn];
-            tok = slot / P.k;
-            wgt = P.topk_w[slot];
-          }
-          atomicAdd(&oacc[tok * kTileRows + g], wgt * (acc[q] * fa));
-          atomicAdd(&oacc[tok * kTileRows + g + 8], wgt * (acc[2 + q] * fb));
-        }
-      }
-    }
-    __syncthreads();  // every warp is done with stage s and the activations
-    if (threadIdx.x == 0 && li + P.stages < nl) issue(list[li + P.stages], s);
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
   }
-  if (!ok) {
-    if (threadIdx.x == 0)
-      for (int s = 0; s < P.stages; ++s) mbar_wait_bounded(&S.bars[s], 0, 1);
+  const int excl = incl - c0 - c1;
+  S.cum[2 * lane] = excl;
+  S.cum[2 * lane + 1] = excl + c0;
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (lane == 0) S.cum[kMaxHit] = total;
+  __syncwarp();
+  for (int e = lane; e < P.E; e += 32) {
+    const uint32_t word = S.bits[e >> 5];
+    const int r = S.rank_base[e >> 5] + __popc(word & ((1u << (e & 31)) - 1u));
+    const bool hit = (word >> (e & 31)) & 1u;
+    P.counts[e] = hit ? S.cnt[r] : 0;
+    P.offsets[e] = r < nh ? S.cum[r] : total;
+  }
+  if (lane == 0) P.offsets[P.E] = total;
+  for (int s = lane; s < Sn; s += 32) {
+    const int e = S.ids[s];
+    if (e < 0) continue;
+    const int r = S.rank_base[e >> 5] + __popc(S.bits[e >> 5] & ((1u << (e & 31)) - 1u));
+    int before = 0;
+    for (int s2 = 0; s2 < s; ++s2) before += S.ids[s2] == e;
+    const int pos = S.cum[r] + before;
+    P.sorted_slot[pos] = s;
+    P.slot_pos[s] = pos;
+  }
+}
+
+constexpr int kRouteWarps = 8;
+constexpr uint32_t kSpinTries = 1u << 20;
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Router scores, one warp per expert, then the last CTA selects. The CTAs do
+// not fence: every score carries the call's tag, and the selecting CTA reads
+// each score until the tag is current. Dynamic shared memory: x rows [T][H]
+// bf16, then the scores [T][E] and the bias [E] (fp32) for the selection.
+__global__ void __launch_bounds__(kRouteWarps * 32) k_dec_route(DecParams P) {
+  extern __shared__ __align__(16) char rsm[];
+  __shared__ RouteSmem S;
+  __shared__ uint32_t tag_s;
+  // The w13 kernel may start now: before it waits for this grid it only reads
+  // the activations and asks L2 for weights.
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!P.layer_mode) {
+    if (warp == 0) build_route_meta(S, P, P.topk_ids, P.topk_w);
     return;
   }
+  const int H = P.H, T = P.T, E = P.E;
+  uint4* xs = reinterpret_cast<uint4*>(rsm);
+  float* ssc = reinterpret_cast<float*>(rsm + size_t(T) * H * 2);
+  float* sbias = ssc + size_t(T) * E;
+  const int e = blockIdx.x * kRouteWarps + warp;
+  // the whole gate row in flight at once (H <= 4096: up to 16 pieces per lane)
+  const uint4* grow = reinterpret_cast<const uint4*>(P.gate + size_t(e < E ? e : 0) * H);
+  const int np = H / 8 / 32;
+  uint4 gv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) gv[i] = i < np ? __ldg(grow + lane + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
+  if (threadIdx.x == 0) tag_s = P.ctl[cEpoch] + 1u;
+  for (int i = threadIdx.x; i < T * H / 8; i += blockDim.x) xs[i] = __ldg(reinterpret_cast<const uint4*>(P.x) + i);
   __syncthreads();
-  for (int i = threadIdx.x; i < T * kTileRows; i += kDThreads) {
-    const int tok = i / kTileRows, r = i % kTileRows;
-    P.out[size_t(tok) * H + m0 + r] = __float2bfloat16_rn(oacc[i]);
+  const uint32_t tag = tag_s;
+  uint64_t* stag = reinterpret_cast<uint64_t*>(P.ctl + cScores);
+  if (e < E)
+    for (int t = 0; t < T; ++t) {
+      const uint4* xrow = xs + size_t(t) * (H / 8);
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < np) {
+          const uint4 xv = xrow[lane + 32 * i];
+          acc = fmaf(bf16_lo(gv[i].x), bf16_lo(xv.x), acc);
+          acc = fmaf(bf16_hi(gv[i].x), bf16_hi(xv.x), acc);
+          acc = fmaf(bf16_lo(gv[i].y), bf16_lo(xv.y), acc);
+          acc = fmaf(bf16_hi(gv[i].y), bf16_hi(xv.y), acc);
+          acc = fmaf(bf16_lo(gv[i].z), bf16_lo(xv.z), acc);
+          acc = fmaf(bf16_hi(gv[i].z), bf16_hi(xv.z), acc);
+          acc = fmaf(bf16_lo(gv[i].w), bf16_lo(xv.w), acc);
+          acc = fmaf(bf16_hi(gv[i].w), bf16_hi(xv.w), acc);
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) stag[size_t(t) * 1024 + e] = (uint64_t(tag) << 32) | __float_as_uint(sqrt_softplus_f(acc));
+    }
+  __syncthreads();
+  if (threadIdx.x == 0) S.is_last = atomicAdd(P.ctl + cTicket, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!S.is_last) return;
+  // ---- the selecting CTA: every score of this call, then the selection
+  bool ok = true;
+  for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
+    const int t = i / E, ee = i % E;
+    const uint64_t* src = stag + size_t(t) * 1024 + ee;
+    uint64_t v = ld_relaxed_u64(src);
+    for (uint32_t k = 0; uint32_t(v >> 32) != tag && k < kSpinTries; ++k) {
+      __nanosleep(32);
+      v = ld_relaxed_u64(src);
+    }
+    ok = ok && uint32_t(v >> 32) == tag;
+    ssc[i] = __uint_as_float(uint32_t(v));
+  }
+  if (!ok) atomicOr(P.status, kStatusTimeout);
+  if (!P.token_ids)
+    for (int i = threadIdx.x; i < E; i += blockDim.x) sbias[i] = __ldg(P.bias + i);
+  __syncthreads();
+  if (warp < T) {
+    if (P.token_ids)
+      select_hash_warp<true>(warp, E, P.k, P.vocab, P.routed_scale, ssc + size_t(warp) * E, P.token_ids, P.tid2eid,
+                             S.sel_ids, S.sel_w, P.status);
+    else if (E <= 256)
+      select_learned_n<false, 8>(warp, E, P.k, P.routed_scale, ssc + size_t(warp) * E, sbias, S.sel_ids, S.sel_w);
+    else
+      select_learned_n<false, 32>(warp, E, P.k, P.routed_scale, ssc + size_t(warp) * E, sbias, S.sel_ids, S.sel_w);
+  }
+  __syncthreads();
+  if (warp == 1)
+    for (int i = lane; i < T * P.k; i += 32) {
+      P.topk_ids[i] = S.sel_ids[i];
+      P.topk_w[i] = S.sel_w[i];
+    }
+  if (warp == 0) {
+    write_permutation(S, P, build_route_meta(S, P, S.sel_ids, S.sel_w));
+    if (lane == 0) {
+      P.ctl[cTicket] = 0u;
+      P.ctl[cEpoch] = tag;
+    }
   }
 }
 
-// x -> decode layout for the forward path that does not go through the fused
-// preparation kernel (routing supplied by the caller).
-__global__ void __launch_bounds__(256) k_dec_xlog(int T, int H, const __nv_bfloat16* __restrict__ x,
-                                                  __half* __restrict__ xlog, int* __restrict__ sigma) {
-  const int warp = threadIdx.x >> 5;
-  const int tt = blockIdx.x * 8 + warp;
-  if (tt < T) warp_row_to_decode_layout(x + size_t(tt) * H, H, xlog + size_t(tt) * H, sigma + tt);
+// ---------------------------------------------------------------- w13 kernel
+
+struct W13Smem {
+  uint64_t full[kStages13];
+  int redcnt[kStages13];
+  int lastfill[kStages13];
+  int sigma[8];
+  uint32_t xmax[2][kGW][8];
+  Tables tb;
+};
+
+constexpr size_t kHead13 = (sizeof(W13Smem) + 127) / 128 * 128;
+constexpr size_t kPart13 = size_t(kStages13) * kGW * 32 * 16;  // float4 per lane and warp
+
+enum Kind : int { kEnd = 0, kS13 = 1, kR13 = 2 };
+struct Item {
+  int kind, li, row0, e;
+};
+
+// Item number -> slab: shared w13 slabs (4 gate + 4 up int8 rows) first, then
+// routed w13 slabs (8 + 8 MXFP4 rows), expert by expert.
+__device__ __forceinline__ Item w13_item(const DecParams& P, const Tables& tb, int it) {
+  Item m = {kEnd, 0, 0, 0};
+  const int n_s = P.Is > 0 ? P.Is / 4 : 0;
+  if (it < n_s) {
+    m.kind = kS13;
+    m.row0 = it * 4;
+  } else {
+    const int r = it - n_s, i8 = P.I / 8;
+    if (r < tb.nh * i8) {
+      m.kind = kR13;
+      m.li = r / i8;
+      m.row0 = (r % i8) * 8;
+      m.e = tb.hit[m.li];
+    }
+  }
+  return m;
 }
 
-size_t w13_fixed(const v4moe_config& c) {
-  return 1024 + size_t((c.n_experts + 1) * 4 + 127) / 128 * 128 + size_t(kDW) * 4 * 32 * 4;
+// Copies slab m into stage s (lane 0 of the calling warp issues and arms).
+__device__ __forceinline__ void fill13(const DecParams& P, W13Smem& S, char* dst, int s, const Item& m, int pos) {
+  const int H = P.H;
+  if ((threadIdx.x & 31) == 0) {
+    S.lastfill[s] = pos;
+    if (m.kind == kS13) {
+      const char* sh = reinterpret_cast<const char*>(P.sh13);
+      mbar_arrive_expect_tx(&S.full[s], uint32_t(8 * H));
+      bulk_g2s(dst, sh + size_t(m.row0) * H, uint32_t(4 * H), &S.full[s]);
+      bulk_g2s(dst + 4 * H, sh + size_t(P.Is + m.row0) * H, uint32_t(4 * H), &S.full[s]);
+    } else {
+      const size_t rg = size_t(m.e) * 2 * P.I + m.row0, ru = rg + P.I;
+      mbar_arrive_expect_tx(&S.full[s], uint32_t(16 * (H / 2) + 16 * (H / 32)));
+      bulk_g2s(dst, P.w13_codes + rg * (H / 2), uint32_t(8 * (H / 2)), &S.full[s]);
+      bulk_g2s(dst + 8 * (H / 2), P.w13_codes + ru * (H / 2), uint32_t(8 * (H / 2)), &S.full[s]);
+      bulk_g2s(dst + 16 * (H / 2), P.w13_scales + rg * (H / 32), uint32_t(8 * (H / 32)), &S.full[s]);
+      bulk_g2s(dst + 16 * (H / 2) + 8 * (H / 32), P.w13_scales + ru * (H / 32), uint32_t(8 * (H / 32)),
+               &S.full[s]);
+    }
+  }
+  __syncwarp();
 }
-size_t w2_fixed(const v4moe_config& c, int T) {
-  return 1024 + size_t((c.n_experts + 2) * 4 + 127) / 128 * 128 + size_t(kDW) * 4 * 32 * 4 +
-         size_t((T * kTileRows * 4 + 127) / 128) * 128;
-}
-int w13_stage(const v4moe_config& c) {
-  return std::max(stage_size(kMx, c.hidden), c.shared_inter > 0 ? stage_size(kS8, c.hidden) : 0);
-}
-int w2_stage(const v4moe_config& c) {
-  return std::max(stage_size(kMx, c.inter), c.shared_inter > 0 ? stage_size(kS8, c.shared_inter) : 0);
-}
-constexpr size_t kSmemMax = 227 * 1024;
 
-// Stages that fit next to the fixed part and the activation rows (up to
-// kMaxStages); `prefer_bytes` caps the size when that still leaves
-// `min_stages` stages (so that two CTAs share an SM).
-void plan(size_t fixed, size_t stage, size_t acts, size_t prefer_bytes, int min_stages, int* stages,
-          size_t* bytes) {
-  const size_t room = kSmemMax > fixed + acts ? kSmemMax - fixed - acts : 0;
-  int s = int(std::min<size_t>(kMaxStages, room / stage));
-  const size_t pref_room = prefer_bytes > fixed + acts ? prefer_bytes - fixed - acts : 0;
-  const int s_pref = int(std::min<size_t>(kMaxStages, pref_room / stage));
-  if (s_pref >= min_stages) s = std::min(s, s_pref);
-  *stages = s;
-  *bytes = fixed + acts + size_t(s) * stage;
+// CTA b's share of the w13 slabs: shared slabs [s0, s1) and routed slabs
+// [r0, r1) (routed slab r is item n_s + r), contiguous so that each expert's
+// rows form one range per CTA. Ring position p is the p-th of these.
+struct Chunk {
+  int s0, s1, r0, r1;
+  __device__ int size() const { return (s1 - s0) + (r1 - r0); }
+  __device__ int item(int p, int n_s) const { return p < s1 - s0 ? s0 + p : n_s + r0 + (p - (s1 - s0)); }
+};
+__device__ __forceinline__ Chunk w13_chunk(const DecParams& P, int nh, int b, int G) {
+  Chunk c;
+  const int n_s = P.Is > 0 ? P.Is / 4 : 0, n_r = nh * (P.I / 8);
+  const int per_s = (n_s + G - 1) / G, per_r = (n_r + G - 1) / G;
+  c.s0 = min(n_s, b * per_s);
+  c.s1 = min(n_s, c.s0 + per_s);
+  c.r0 = min(n_r, b * per_r);
+  c.r1 = min(n_r, c.r0 + per_r);
+  return c;
+}
+
+// Asks L2 for the chunk's shared (routed == false) or routed slabs, as one
+// range per weight tensor and expert (one lane).
+__device__ __forceinline__ void prefetch13(const DecParams& P, const Tables& tb, const Chunk& c, bool routed) {
+  const int H = P.H;
+  if (!routed) {
+    if (c.s1 <= c.s0) return;
+    const char* sh = reinterpret_cast<const char*>(P.sh13);
+    prefetch_l2_range(sh + size_t(4 * c.s0) * H, size_t(4 * (c.s1 - c.s0)) * H);
+    prefetch_l2_range(sh + size_t(P.Is + 4 * c.s0) * H, size_t(4 * (c.s1 - c.s0)) * H);
+    return;
+  }
+  const int i8 = P.I / 8;
+  for (int r = c.r0; r < c.r1;) {
+    const int li = r / i8, re = min(c.r1, (li + 1) * i8);
+    const size_t rows = size_t(8) * (re - r);
+    const size_t rg = size_t(tb.hit[li]) * 2 * P.I + size_t(8) * (r - li * i8), ru = rg + P.I;
+    prefetch_l2_range(P.w13_codes + rg * (H / 2), rows * (H / 2));
+    prefetch_l2_range(P.w13_codes + ru * (H / 2), rows * (H / 2));
+    prefetch_l2_range(P.w13_scales + rg * (H / 32), rows * (H / 32));
+    prefetch_l2_range(P.w13_scales + ru * (H / 32), rows * (H / 32));
+    r = re;
+  }
+}
+
+// The w2 rows of the 16-row output blocks that CTA b of the w2 kernel owns
+// (blocks [b w2_per, (b + 1) w2_per)): the shared expert's, or every routed
+// expert's (one lane).
+__device__ __forceinline__ void prefetch_w2_share(const DecParams& P, const Tables& tb, int b, bool routed) {
+  const int nrb = P.H / 16;
+  const int rb0 = min(nrb, b * P.w2_per), rb1 = min(nrb, rb0 + P.w2_per);
+  if (rb1 <= rb0) return;
+  const size_t rows = size_t(16) * (rb1 - rb0);
+  if (!routed) {
+    if (P.Is > 0) prefetch_l2_range(reinterpret_cast<const char*>(P.sh2) + size_t(16 * rb0) * P.Is, rows * P.Is);
+    return;
+  }
+  for (int li = 0; li < tb.nh; ++li) {
+    const size_t r0 = size_t(tb.hit[li]) * P.H + size_t(16) * rb0;
+    prefetch_l2_range(P.w2_codes + r0 * (P.I / 2), rows * (P.I / 2));
+    prefetch_l2_range(P.w2_scales + r0 * (P.I / 32), rows * (P.I / 32));
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
+  extern __shared__ __align__(128) char smem[];
+  W13Smem& S = *reinterpret_cast<W13Smem*>(smem);
+  char* stages = smem + kHead13;
+  float4* parts = reinterpret_cast<float4*>(stages + size_t(kStages13) * P.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = P.T, H = P.H;
+  const int G = int(gridDim.x), b = int(blockIdx.x);
+  const int n_s = P.Is > 0 ? P.Is / 4 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages13; ++s) {
+      mbar_init(&S.full[s], 1);
+      S.redcnt[s] = 0;
+      S.lastfill[s] = -1;
+    }
+    S.tb.nh = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // The w2 kernel may launch now (its CTAs start as these leave their SMs).
+  pdl_launch_dependents();
+  // Ask L2 for everything that does not depend on the routing.
+  if (warp == 15 && lane == 0) {
+    prefetch13(P, S.tb, w13_chunk(P, 0, b, G), false);
+    prefetch_w2_share(P, S.tb, b, false);
+  }
+
+  const int q = warp / kGW, wi = warp % kGW;
+  const int g = lane >> 2, t = lane & 3;
+  const int nkbH = H / 128;
+  // ---- x slices of this warp's K blocks for token g, then f16 scaled by 2^sigma
+  uint32_t B[kNJ][16];
+  uint32_t mx = 0u;
+#pragma unroll
+  for (int j = 0; j < kNJ; ++j) {
+    const int kb = wi + 8 * j;
+    if (kb < nkbH && g < T) {
+      const uint4* src = reinterpret_cast<const uint4*>(P.x + size_t(g) * H + kb * 128 + 32 * t);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const uint4 v = __ldg(src + p);
+        B[j][4 * p] = v.x;
+        B[j][4 * p + 1] = v.y;
+        B[j][4 * p + 2] = v.z;
+        B[j][4 * p + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) B[j][i] = 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mx = absmax_bf16x2(mx, B[j][i]);
+  }
+  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  if (t == 0) S.xmax[q][wi][g] = mx;
+  named_bar_sync(2 + q, kGW * 32);
+  {
+    uint32_t rmx = 0u;
+    for (int w = 0; w < kGW; ++w) rmx = max(rmx, S.xmax[q][w][g]);
+    const int sg = sigma_of(rmx);
+    if (warp == 0 && t == 0) S.sigma[g] = sg;
+    const float mul = __int_as_float((sg + 127) << 23);
+#pragma unroll
+    for (int j = 0; j < kNJ; ++j)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const __half2 hv = __floats2half2_rn(bf16_lo(B[j][i]) * mul, bf16_hi(B[j][i]) * mul);
+        B[j][i] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+  }
+
+  // ---- the routing (previous grid) is complete and visible past this point
+  pdl_wait();
+  read_tables(S.tb, P);
+  __syncthreads();
+  const Chunk ch = w13_chunk(P, S.tb.nh, b, G);
+  const int npos = ch.size();
+  // The routed slabs stream through the ring; the routed w2 rows of this CTA's
+  // share are asked for once its last slab is on its way.
+  if (warp == 14) {
+    for (int p = 0; p < kStages13 && p < npos; ++p)
+      fill13(P, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, ch.item(p, n_s)), p);
+    if (npos <= kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
+  }
+
+  // ---- item loop: group q takes ring positions q, q + 2, ...
+  for (int pos = q; pos < npos; pos += 2) {
+    const Item m = w13_item(P, S.tb, ch.item(pos, n_s));
+    const int s = pos % kStages13;
+    if (!__all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / kStages13) & 1u, P))) break;
+    const char* st = stages + size_t(s) * P.stage_bytes;
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 p0;
+    if (m.kind == kR13) {
+      const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + 16 * (H / 2));
+      float fa, fb;
+      tile_mx<kNJ, 8>(st + g * (H / 2), st + (g + 8) * (H / 2), sc + g * (H / 32), sc + (g + 8) * (H / 32), wi,
+                      nkbH, B, a0, a1, fa, fb);
+      p0 = make_float4((a0[0] + a1[0]) * fa, (a0[1] + a1[1]) * fa, (a0[2] + a1[2]) * fb, (a0[3] + a1[3]) * fb);
+    } else {
+      // rows g < 4: gate row g of the slab (tile row g) and up row g (tile row g + 8)
+      tile_s8<kNJ, 8>(st + (g & 3) * H, st + (4 + (g & 3)) * H, g < 4, 0, nkbH, wi, B, a0, a1);
+      p0 = make_float4(a0[0] + a1[0], a0[1] + a1[1], a0[2] + a1[2], a0[3] + a1[3]);
+    }
+    float4* part = parts + size_t(s) * kGW * 32;
+    part[wi * 32 + lane] = p0;
+    __threadfence_block();
+    __syncwarp();
+    int old = 0;
+    if (lane == 0) old = atomicAdd(&S.redcnt[s], 1);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != kGW - 1) continue;
+    // Last of the group: the stage and its partials are this warp's alone.
+    __threadfence_block();
+    float4 d = part[lane];
+#pragma unroll
+    for (int w = 1; w < kGW; ++w) {
+      const float4 v = part[w * 32 + lane];
+      d.x += v.x;
+      d.y += v.y;
+      d.z += v.z;
+      d.w += v.w;
+    }
+    if (lane == 0) S.redcnt[s] = 0;
+    __syncwarp();
+    if (pos + kStages13 < npos) {
+      fill13(P, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, ch.item(pos + kStages13, n_s)),
+             pos + kStages13);
+      if (pos + kStages13 == npos - 1 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
+    }
+    const float dg[2] = {d.x, d.y}, du[2] = {d.z, d.w};
+    if (m.kind == kR13) {
+      const uint32_t mask = S.tb.mask[m.li];
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int tok = 2 * t + qq;
+        if (tok < T && ((mask >> tok) & 1u)) {
+          const float inv = pow2f(-S.sigma[tok]);
+          const float h = clamped_swiglu_f(dg[qq] * inv, du[qq] * inv, P.limit) * S.tb.w[m.li * 8 + tok];
+          P.dh[(size_t(m.li) * T + tok) * P.I + m.row0 + g] = __float2half_rn(h);
+        }
+      }
+    } else if (g < 4) {
+      const float sg = __ldg(P.sh13_scale + m.row0 + g), su = __ldg(P.sh13_scale + P.Is + m.row0 + g);
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int tok = 2 * t + qq;
+        if (tok < T) {
+          const float inv = pow2f(-S.sigma[tok]);
+          P.hs[size_t(tok) * P.Is + m.row0 + g] =
+              __float2half_rn(clamped_swiglu_f(dg[qq] * sg * inv, du[qq] * su * inv, P.limit));
+        }
+      }
+    }
+  }
+  // No copy may still be landing in this CTA's shared memory (possible only
+  // after a timeout).
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int s = 0; s < kStages13; ++s)
+      if (S.lastfill[s] >= 0) mbar_wait_bounded(&S.full[s], uint32_t(S.lastfill[s] / kStages13) & 1u, kBarTries);
+}
+
+// ---------------------------------------------------------------- w2 kernel
+
+struct W2Smem {
+  uint64_t full[kMaxStages2];
+  int redcnt[kMaxStages2];
+  int lastfill[kMaxStages2];
+  Tables tb;
+};
+constexpr size_t kHead2 = (sizeof(W2Smem) + 127) / 128 * 128;
+constexpr size_t kRed2 = size_t(16) * 32 * 16;  // float4 per lane and warp
+
+// Ring position p of CTA b: output block rb = b w2_per + p / nl, expert slot
+// l = p % nl (the shared expert first when there is one, then the routed list).
+struct Item2 {
+  int rb, l, li;  // li < 0: shared expert
+};
+__device__ __forceinline__ Item2 w2_item(const DecParams& P, int nl, int b, int p) {
+  Item2 m;
+  m.rb = b * P.w2_per + p / nl;
+  m.l = p % nl;
+  m.li = P.Is > 0 ? m.l - 1 : m.l;
+  return m;
+}
+
+// Offset of the token rows of intermediates in a stage.
+__device__ __forceinline__ int w2_hoff(const DecParams& P) {
+  return max(16 * P.Is, 16 * (P.I / 2) + 16 * (P.I / 32));
+}
+
+// Weight rows [rb * 16, +16) of the item's expert: adds their bytes to the
+// stage's barrier without arriving (lane 0).
+__device__ __forceinline__ void fill2_weights(const DecParams& P, W2Smem& S, char* dst, int s, const Item2& m) {
+  if (m.li < 0) {
+    mbar_expect_tx(&S.full[s], uint32_t(16 * P.Is));
+    bulk_g2s(dst, reinterpret_cast<const char*>(P.sh2) + size_t(m.rb) * 16 * P.Is, uint32_t(16 * P.Is), &S.full[s]);
+  } else {
+    const size_t r0 = size_t(S.tb.hit[m.li]) * P.H + size_t(m.rb) * 16;
+    mbar_expect_tx(&S.full[s], uint32_t(16 * (P.I / 2) + 16 * (P.I / 32)));
+    bulk_g2s(dst, P.w2_codes + r0 * (P.I / 2), uint32_t(16 * (P.I / 2)), &S.full[s]);
+    bulk_g2s(dst + 16 * (P.I / 2), P.w2_scales + r0 * (P.I / 32), uint32_t(16 * (P.I / 32)), &S.full[s]);
+  }
+}
+
+// The intermediates of the expert's tokens (token t in slot t), then the
+// stage's one arrival (whole warp). Only after the w13 grid is complete.
+__device__ __forceinline__ void fill2_h(const DecParams& P, W2Smem& S, char* dst, int s, const Item2& m) {
+  const int lane = threadIdx.x & 31;
+  const bool sh = m.li < 0;
+  const int K = sh ? P.Is : P.I;
+  const uint32_t mask = sh ? (1u << P.T) - 1u : S.tb.mask[m.li];
+  if (lane == 0) mbar_arrive_expect_tx(&S.full[s], uint32_t(__popc(mask)) * uint32_t(K * 2));
+  __syncwarp();
+  if (lane < P.T && ((mask >> lane) & 1u)) {
+    const __half* src = sh ? P.hs + size_t(lane) * P.Is : P.dh + (size_t(m.li) * P.T + lane) * P.I;
+    bulk_g2s(dst + w2_hoff(P) + lane * K * 2, src, uint32_t(K * 2), &S.full[s]);
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
+  extern __shared__ __align__(128) char smem[];
+  W2Smem& S = *reinterpret_cast<W2Smem*>(smem);
+  char* stages = smem + kHead2;
+  float4* red = reinterpret_cast<float4*>(stages + size_t(P.nstages) * P.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int T = P.T, NS = P.nstages;
+  const int b = int(blockIdx.x);
+  const int nrb_mine = max(0, min(P.w2_per, P.H / 16 - b * P.w2_per));
+  const bool has_sh = P.Is > 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&S.full[s], 1);
+      S.redcnt[s] = 0;
+      S.lastfill[s] = -1;
+    }
+    fence_mbar_init();
+    // Position 0 is the shared expert of the first block: its weight rows do
+    // not depend on the previous grids.
+    if (has_sh && nrb_mine > 0) fill2_weights(P, S, stages, 0, Item2{b * P.w2_per, 0, -1});
+  }
+  __syncthreads();
+  pdl_wait();
+  read_tables(S.tb, P);
+  __syncthreads();
+  const int nl = S.tb.nh + (has_sh ? 1 : 0);
+  const int n_items = nrb_mine * nl;
+  if (warp == 0)
+    for (int p = 0; p < NS && p < n_items; ++p) {
+      const Item2 m = w2_item(P, nl, b, p);
+      if (lane == 0) {
+        S.lastfill[p] = p;
+        if (!(p == 0 && has_sh)) fill2_weights(P, S, stages + size_t(p) * P.stage_bytes, p, m);
+      }
+      __syncwarp();
+      fill2_h(P, S, stages + size_t(p) * P.stage_bytes, p, m);
+    }
+  // Position 0's shared weights were armed before the wait even if it turns
+  // out there is nothing to do; give that copy its arrival so it can land.
+  if (warp == 0 && n_items == 0 && has_sh && nrb_mine > 0 && lane == 0) {
+    S.lastfill[0] = 0;
+    mbar_arrive(&S.full[0]);
+  }
+
+  bool ok = true;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int pos = 0; pos < n_items; ++pos) {
+    const Item2 m = w2_item(P, nl, b, pos);
+    const int s = pos % NS;
+    // A timed-out warp keeps going (without reading the stage) so that every
+    // warp reaches the block-end barriers.
+    ok = ok && __all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / NS) & 1u, P));
+    const char* st = stages + size_t(s) * P.stage_bytes;
+    const bool sh = m.li < 0;
+    const int K = sh ? P.Is : P.I;
+    const int nkb = K / 128;
+    if (ok) {
+      // B: the intermediates of token g (zero for tokens not routed here)
+      const uint32_t mask = sh ? (1u << T) - 1u : S.tb.mask[m.li];
+      const bool has_tok = g < T && ((mask >> g) & 1u);
+      uint32_t Bf[2][16];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int kb = warp + 16 * j;
+        if (has_tok && kb < nkb) {
+          const uint4* p4 = reinterpret_cast<const uint4*>(st + w2_hoff(P) + g * K * 2 + kb * 256 + 64 * t);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const uint4 v = p4[p];
+            Bf[j][4 * p] = v.x;
+            Bf[j][4 * p + 1] = v.y;
+            Bf[j][4 * p + 2] = v.z;
+            Bf[j][4 * p + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) Bf[j][i] = 0u;
+        }
+      }
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (sh) {
+        tile_s8<2, 16>(st + g * P.Is, st + (g + 8) * P.Is, true, 0, nkb, warp, Bf, a0, a1);
+        const float sa = __ldg(P.sh2_scale + m.rb * 16 + g), sb = __ldg(P.sh2_scale + m.rb * 16 + g + 8);
+        acc.x += (a0[0] + a1[0]) * sa;
+        acc.y += (a0[1] + a1[1]) * sa;
+        acc.z += (a0[2] + a1[2]) * sb;
+        acc.w += (a0[3] + a1[3]) * sb;
+      } else {
+        const int rs = P.I / 2, Gs = P.I / 32;
+        const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + 16 * rs);
+        float fa, fb;
+        tile_mx<2, 16>(st + g * rs, st + (g + 8) * rs, sc + g * Gs, sc + (g + 8) * Gs, warp, nkb, Bf, a0, a1, fa,
+                       fb);
+        acc.x += (a0[0] + a1[0]) * fa;
+        acc.y += (a0[1] + a1[1]) * fa;
+        acc.z += (a0[2] + a1[2]) * fb;
+        acc.w += (a0[3] + a1[3]) * fb;
+      }
+      // the last warp to finish with the stage refills it
+      __syncwarp();
+      int old = 0;
+      if (lane == 0) old = atomicAdd(&S.redcnt[s], 1);
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (old == 15) {
+        if (lane == 0) S.redcnt[s] = 0;
+        __syncwarp();
+        const int np = pos + NS;
+        if (np < n_items) {
+          const Item2 mn = w2_item(P, nl, b, np);
+          if (lane == 0) {
+            S.lastfill[s] = np;
+            fill2_weights(P, S, stages + size_t(s) * P.stage_bytes, s, mn);
+          }
+          __syncwarp();
+          fill2_h(P, S, stages + size_t(s) * P.stage_bytes, s, mn);
+        }
+      }
+    }
+    if (m.l == nl - 1) {
+      // block done: sum the 16 warps' partials in warp order, write bf16
+      red[warp * 32 + lane] = acc;
+      __syncthreads();
+      if (warp == 0) {
+        float4 d = red[lane];
+        for (int w = 1; w < 16; ++w) {
+          const float4 v = red[w * 32 + lane];
+          d.x += v.x;
+          d.y += v.y;
+          d.z += v.z;
+          d.w += v.w;
+        }
+        const float v[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tok = 2 * t + (i & 1);
+          if (tok < T) P.out[size_t(tok) * P.H + m.rb * 16 + g + 8 * (i >> 1)] = __float2bfloat16_rn(v[i]);
+        }
+      }
+      __syncthreads();
+      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  if (nl == 0) {  // nothing contributes: the output is zero
+    for (int i = threadIdx.x; i < nrb_mine * 16 * T; i += blockDim.x) {
+      const int r = i / (16 * T), rem = i % (16 * T);
+      P.out[size_t(rem / 16) * P.H + (b * P.w2_per + r) * 16 + rem % 16] = __float2bfloat16_rn(0.f);
+    }
+  }
+  // No copy may still be landing in this CTA's shared memory.
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int s = 0; s < NS; ++s)
+      if (S.lastfill[s] >= 0) mbar_wait_bounded(&S.full[s], uint32_t(S.lastfill[s] / NS) & 1u, kBarTries);
+}
+
+// ---------------------------------------------------------------- host side
+
+struct Plan {
+  int stage13 = 0, stage2 = 0, nst2 = 0;
+  size_t smem13 = 0, smem2 = 0;
+  bool ok = false;
+};
+
+Plan make_plan(const v4moe_config& c, int T) {
+  Plan p;
+  if (T < 1 || T > kDecodeMaxTokens || T * c.top_k > kMaxHit) return p;
+  const int H = c.hidden, I = c.inter, Is = c.shared_inter;
+  if (H > kNJ * 8 * 128 || I > 2 * 16 * 128 || Is > 2 * 16 * 128) return p;
+  int s13 = 16 * (H / 2) + 16 * (H / 32);
+  if (Is > 0) s13 = std::max(s13, 8 * H);
+  p.stage13 = (s13 + 127) / 128 * 128;
+  p.smem13 = kHead13 + size_t(kStages13) * p.stage13 + kPart13;
+  const int hoff = std::max(16 * Is, 16 * (I / 2) + 16 * (I / 32));
+  const int s2 = hoff + T * std::max(I, Is) * 2;
+  p.stage2 = (s2 + 127) / 128 * 128;
+  const size_t room = 227 * 1024 - kHead2 - kRed2;
+  p.nst2 = int(std::min<size_t>(kMaxStages2, room / p.stage2));
+  p.smem2 = kHead2 + size_t(p.nst2) * p.stage2 + kRed2;
+  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2;
+  return p;
 }
 
 }  // namespace
 
-bool dec_supported(const v4moe_config& c, int T) {
-  if (T > kDecodeMaxTokens || T < 1) return false;
-  int s13, s2;
-  size_t b13, b2;
-  plan(w13_fixed(c), w13_stage(c), size_t(T) * xs_stride(c.hidden), kSmemMax, 2, &s13, &b13);
-  plan(w2_fixed(c, T), w2_stage(c), size_t(T) * xs_stride(std::max(c.inter, c.shared_inter)), kSmemMax, 2,
-       &s2, &b2);
-  return s13 >= 2 && s2 >= 2;
+DecodeBuffers dec_buffers(const v4moe_config& c, int64_t T) {
+  DecodeBuffers b;
+  if (T < 1 || T > kDecodeMaxTokens) return b;
+  b.ctl = size_t(cWords) * 4;
+  b.dh = size_t(kMaxHit) * T * c.inter * 2;
+  b.hs = size_t(T) * std::max(c.shared_inter, 0) * 2;
+  return b;
 }
 
-cudaError_t launch_dec_xlog(const v4moe_config& c, int T, const __nv_bfloat16* x, __half* xlog, int* sigma,
-                            cudaStream_t st) {
-  return launch_kernel("dec_xlog", k_dec_xlog, dim3((T + 7) / 8), dim3(256), 0, st, false, T, c.hidden, x, xlog,
-                       sigma);
-}
+bool dec_supported(const v4moe_config& c, int T) { return make_plan(c, T).ok; }
 
-cudaError_t launch_forward_dec(const ForwardArgs& a, const __half* xlog, const int* sigma, cudaStream_t st) {
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const v4moe_config& c = a.c;
-  if (a.T == 0) return cudaSuccess;
+  const Plan p = make_plan(c, a.T);
+  if (!p.ok) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   DecParams P;
   P.T = a.T;
   P.H = c.hidden;
@@ -589,12 +1032,25 @@ cudaError_t launch_forward_dec(const ForwardArgs& a, const __half* xlog, const i
   P.Is = c.shared_inter;
   P.E = c.n_experts;
   P.k = c.top_k;
+  P.vocab = c.vocab;
   P.limit = c.swiglu_limit;
-  P.xlog = xlog;
-  P.sigma = sigma;
+  P.routed_scale = c.routed_scale;
+  P.layer_mode = a.layer_mode;
+  P.stage_bytes = 0;
+  P.nstages = 0;
+  P.w2_per = 1;
+  P.x = a.x;
+  P.gate = a.gate;
+  P.bias = a.bias;
+  P.token_ids = a.token_ids;
+  P.tid2eid = a.tid2eid;
+  P.topk_ids = a.topk_ids;
+  P.topk_w = a.topk_w;
+  P.counts = a.counts;
   P.offsets = a.offsets;
   P.sorted_slot = a.sorted_slot;
-  P.topk_w = a.topk_w;
+  P.slot_pos = a.slot_pos;
+  P.scores = a.scores;
   P.w13_codes = a.w.w13_codes;
   P.w13_scales = a.w.w13_scales;
   P.w2_codes = a.w.w2_codes;
@@ -603,43 +1059,30 @@ cudaError_t launch_forward_dec(const ForwardArgs& a, const __half* xlog, const i
   P.sh13_scale = a.w.sh_w13_scale;
   P.sh2 = a.w.sh_w2;
   P.sh2_scale = a.w.sh_w2_scale;
-  P.hlog = reinterpret_cast<__half*>(a.h);
-  P.hslog = reinterpret_cast<__half*>(a.hs);
-  P.out = a.out;
+  P.dh = a.dh;
+  P.hs = a.hs;
+  P.ctl = a.ctl;
   P.status = a.status;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  P.out = a.out;
 
-  // ---- w13: one persistent CTA per SM; a share of them on the shared expert,
-  // sized by its fraction of the weight bytes (routed experts hit <= T*k).
-  int stages13;
-  size_t smem13;
-  plan(w13_fixed(c), w13_stage(c), size_t(a.T) * xs_stride(c.hidden), kSmemMax, 2, &stages13, &smem13);
-  const int grid13 = sms;
-  int nsh = 0;
-  if (c.shared_inter > 0) {
-    const double sh_bytes = double(2 * c.shared_inter) * c.hidden;
-    const double rt_bytes = double(std::min(c.n_experts, a.T * c.top_k)) * (2.0 * c.inter * c.hidden / 2);
-    nsh = int(std::lround(grid13 * sh_bytes / (sh_bytes + rt_bytes)));
-    nsh = std::max(1, std::min(grid13 - 1, nsh));
-  }
-  P.n_shared_ctas = nsh;
-  P.stages = stages13;
-  P.stage_bytes = w13_stage(c);
-  set_smem(k_dec_w13, smem13);
-  cudaError_t e = launch_kernel("dec_w13", k_dec_w13, dim3(grid13), dim3(kDThreads), smem13, st, true, P);
+  const int nrb = c.hidden / 16;
+  P.w2_per = (nrb + sms - 1) / sms;
+  const int grid2 = (nrb + P.w2_per - 1) / P.w2_per;
+  const int route_grid = a.layer_mode ? (c.n_experts + kRouteWarps - 1) / kRouteWarps : 1;
+  const size_t route_smem =
+      a.layer_mode ? size_t(a.T) * c.hidden * 2 + size_t(a.T) * c.n_experts * 4 + size_t(c.n_experts) * 4 : 0;
+  set_smem(k_dec_route, route_smem);
+  cudaError_t e =
+      launch_kernel("dec_route", k_dec_route, dim3(route_grid), dim3(kRouteWarps * 32), route_smem, st, false, P);
   if (e != cudaSuccess) return e;
-
-  // ---- w2 + combine: one CTA per 16 output rows; aim for two CTAs per SM.
-  int stages2;
-  size_t smem2;
-  plan(w2_fixed(c, a.T), w2_stage(c), size_t(a.T) * xs_stride(std::max(c.inter, c.shared_inter)),
-       kSmemMax / 2 - 1024, 3, &stages2, &smem2);
-  P.stages = stages2;
-  P.stage_bytes = w2_stage(c);
-  set_smem(k_dec_w2, smem2);
-  return launch_kernel("dec_w2", k_dec_w2, dim3(c.hidden / kTileRows), dim3(kDThreads), smem2, st, true, P);
+  P.stage_bytes = p.stage13;
+  set_smem(k_dec_w13, p.smem13);
+  e = launch_kernel("dec_w13", k_dec_w13, dim3(sms), dim3(kThreads), p.smem13, st, true, P);
+  if (e != cudaSuccess) return e;
+  P.stage_bytes = p.stage2;
+  P.nstages = p.nst2;
+  set_smem(k_dec_w2, p.smem2);
+  return launch_kernel("dec_w2", k_dec_w2, dim3(grid2), dim3(kThreads), p.smem2, st, true, P);
 }
 
 }  // namespace v4moe

@@ -35,31 +35,40 @@ __device__ __forceinline__ void sort8_by_id(int id[8], float v[8]) {
   }
 }
 
+// Order-preserving map of a float to an unsigned key (larger float, larger key).
+__device__ __forceinline__ uint32_t float_key(float v) {
+  const uint32_t b = __float_as_uint(v);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // Learned routing of token t from its E scores s (fp32; SCORE_L2 reads them
 // through L2, for scores written by other CTAs of the same kernel): k rounds
-// of a warp arg-max over s + bias (largest value, then lowest id) that carry
-// the unbiased score along; ids written in ascending order; w = scale * s[id]
-// / sum of the selected s. Every load is issued before the first use.
-template <bool SCORE_L2>
-__device__ __forceinline__ void select_learned(int t, int E, int k, float routed_scale, const float* s,
-                                               const float* __restrict__ bias, int32_t* __restrict__ topk_ids,
-                                               float* __restrict__ topk_w) {
+// of a warp arg-max over s + bias (largest value, then lowest id), each round
+// two warp reductions (largest key, then lowest id holding it); the winner's
+// unbiased score comes from its lane. Ids are written in ascending order; w =
+// scale * s[id] / sum of the selected s. Every load is issued before the first
+// use. NPER bounds the experts per lane (E <= 32 * NPER).
+template <bool SCORE_L2, int NPER>
+__device__ __forceinline__ void select_learned_n(int t, int E, int k, float routed_scale, const float* s,
+                                                 const float* bias, int32_t* __restrict__ topk_ids,
+                                                 float* __restrict__ topk_w) {
   const int lane = threadIdx.x & 31;
   const int nper = (E + 31) / 32;
-  float sv[32], b[32];
+  float sv[NPER], b[NPER];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NPER; ++i) {
     const int e = lane + 32 * i;
     const int ec = (i < nper && e < E) ? e : 0;
     sv[i] = SCORE_L2 ? __ldcg(s + ec) : s[ec];
-    b[i] = __ldg(bias + ec);
+    b[i] = bias[ec];  // global or shared
   }
+  // key 0: not an expert; a NaN sum ranks as -inf
+  uint32_t key[NPER];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NPER; ++i) {
     const int e = lane + 32 * i;
-    float v = sv[i] + b[i];
-    if (!(i < nper && e < E) || v != v) v = -INFINITY;  // NaN never wins
-    b[i] = v;
+    const float v = sv[i] + b[i];
+    key[i] = (i < nper && e < E) ? float_key(v != v ? -INFINITY : v) : 0u;
   }
   uint32_t taken = 0;
   int id[8];
@@ -69,31 +78,23 @@ __device__ __forceinline__ void select_learned(int t, int E, int k, float routed
     id[r] = 0x7fffffff;
     sel[r] = 0.0f;
     if (r < k) {
-      float bv = -INFINITY, sb = 0.0f;
-      int be = 0x7fffffff;
+      uint32_t lk = 0u;
+      int li = 0;
+      float ls = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int e = lane + 32 * i;
-        if (i < nper && e < E && !((taken >> i) & 1u) && (b[i] > bv || be == 0x7fffffff)) {
-          bv = b[i];
-          be = e;
-          sb = sv[i];
+      for (int i = 0; i < NPER; ++i)
+        if (!((taken >> i) & 1u) && key[i] > lk) {  // strict: lowest id among equal keys
+          lk = key[i];
+          li = i;
+          ls = sv[i];
         }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        const float os = __shfl_xor_sync(0xffffffffu, sb, o);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-          sb = os;
-        }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      id[r] = be;
-      sel[r] = sb;
+      const uint32_t mk = __reduce_max_sync(0xffffffffu, lk);
+      const uint32_t cand = (lk == mk && lk != 0u) ? uint32_t(lane + 32 * li) : 0xffffffffu;
+      const uint32_t wid = __reduce_min_sync(0xffffffffu, cand);
+      const float ws = __shfl_sync(0xffffffffu, ls, int(wid & 31u));
+      if (lane == int(wid & 31u)) taken |= 1u << (wid >> 5);
+      id[r] = int(wid);
+      sel[r] = ws;
     }
   }
   sort8_by_id(id, sel);
@@ -112,6 +113,16 @@ __device__ __forceinline__ void select_learned(int t, int E, int k, float routed
     topk_ids[size_t(t) * k + lane] = myid;
     topk_w[size_t(t) * k + lane] = routed_scale * (myv / sum);
   }
+}
+
+template <bool SCORE_L2>
+__device__ __forceinline__ void select_learned(int t, int E, int k, float routed_scale, const float* s,
+                                               const float* __restrict__ bias, int32_t* __restrict__ topk_ids,
+                                               float* __restrict__ topk_w) {
+  if (E <= 256)
+    select_learned_n<SCORE_L2, 8>(t, E, k, routed_scale, s, bias, topk_ids, topk_w);
+  else
+    select_learned_n<SCORE_L2, 32>(t, E, k, routed_scale, s, bias, topk_ids, topk_w);
 }
 
 // Hash routing of token t (first layers: "select experts from a token-id hash

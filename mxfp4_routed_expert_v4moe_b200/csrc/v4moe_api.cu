@@ -156,6 +156,25 @@ ForwardArgs forward_args(const v4moe_config* cfg, int32_t T, const void* x, cons
   return a;
 }
 
+// Arguments of the single-kernel decode path; routing pointers are filled in
+// by the caller for layer mode.
+DecodeArgs decode_args(const v4moe_config* cfg, int32_t T, const void* x, const v4moe_weights* weights, void* out,
+                       void* ws) {
+  const WsLayout L = ws_layout(*cfg, T);
+  DecodeArgs d = {};
+  d.c = *cfg;
+  d.T = T;
+  d.x = static_cast<const __nv_bfloat16*>(x);
+  d.w = *weights;
+  d.out = static_cast<__nv_bfloat16*>(out);
+  d.status = at<uint32_t>(ws, L.status);
+  d.scores = at<float>(ws, L.scores);
+  d.ctl = at<uint32_t>(ws, L.d_ctl);
+  d.dh = at<__half>(ws, L.d_dh);
+  d.hs = at<__half>(ws, L.d_hs);
+  return d;
+}
+
 }  // namespace
 }  // namespace v4moe
 
@@ -177,14 +196,15 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x, const i
   if (int32_t r = check_device()) return r;
   if (T == 0) return V4MOE_OK;
   const WsLayout L = ws_layout(*cfg, T);
-  const ForwardArgs a = forward_args(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, weights, out, ws);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dec_supported(*cfg, T)) {
-    __half* xlog = at<__half>(ws, L.xlog);
-    int* sigma = at<int>(ws, L.sigma);
-    if (cudaError_t e = launch_dec_xlog(*cfg, T, a.x, xlog, sigma, st)) return launch_status(e);
-    return launch_status(launch_forward_dec(a, xlog, sigma, st));
+    DecodeArgs d = decode_args(cfg, T, x, weights, out, ws);
+    d.layer_mode = 0;
+    d.topk_ids = const_cast<int32_t*>(topk_ids);
+    d.topk_w = const_cast<float*>(topk_w);
+    return launch_status(launch_decode(d, st));
   }
+  const ForwardArgs a = forward_args(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, weights, out, ws);
   return launch_status(launch_forward_tc(a, at<__half>(ws, L.xlog), at<int>(ws, L.sigma), at<char>(ws, L.tc), st));
 }
 
@@ -207,20 +227,20 @@ int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const voi
   if (int32_t r = check_device()) return r;
   // an empty batch still reports empty counts and offsets
   if (T == 0) return v4moe_permute(cfg, 0, topk_ids, counts, offsets, sorted_slot, slot_pos, ws, ws_bytes, stream);
-  const WsLayout L = ws_layout(*cfg, T);
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (dec_supported(*cfg, T)) {
-    __half* xlog = at<__half>(ws, L.xlog);
-    int* sigma = at<int>(ws, L.sigma);
-    uint32_t* status = at<uint32_t>(ws, L.status);
-    if (cudaError_t e = launch_dec_prep(*cfg, T, xb, static_cast<const __nv_bfloat16*>(gate), bias, token_ids,
-                                        tid2eid, topk_ids, topk_w, counts, offsets, sorted_slot, slot_pos,
-                                        at<float>(ws, L.scores), xlog, sigma, status,
-                                        reinterpret_cast<unsigned*>(status + kTicketWord), st))
-      return launch_status(e);
-    const ForwardArgs a = forward_args(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, weights, out, ws);
-    return launch_status(launch_forward_dec(a, xlog, sigma, st));
+    DecodeArgs d = decode_args(cfg, T, x, weights, out, ws);
+    d.layer_mode = 1;
+    d.gate = static_cast<const __nv_bfloat16*>(gate);
+    d.bias = bias;
+    d.token_ids = token_ids;
+    d.tid2eid = tid2eid;
+    d.topk_ids = topk_ids;
+    d.topk_w = topk_w;
+    d.counts = counts;
+    d.offsets = offsets;
+    d.sorted_slot = sorted_slot;
+    d.slot_pos = slot_pos;
+    return launch_status(launch_decode(d, static_cast<cudaStream_t>(stream)));
   }
   if (int32_t r = v4moe_route(cfg, T, x, gate, bias, token_ids, tid2eid, topk_ids, topk_w, ws, ws_bytes, stream))
     return r;

@@ -11,8 +11,7 @@
 namespace v4moe {
 
 // Status block (first 256 bytes of the workspace): word 0 is the device
-// status word, word 1 the ticket of the fused decode preparation kernel.
-constexpr size_t kTicketWord = 1;
+// status word.
 // Device status word bits.
 constexpr uint32_t kStatusBadExpertId = 1u << 0;
 constexpr uint32_t kStatusBadTokenId = 1u << 1;
@@ -25,6 +24,13 @@ inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a
 constexpr int kPermChunk = 2048;
 
 size_t tc_extra_bytes(const v4moe_config& c, int64_t T);
+
+// Buffers of the decode path (all zero bytes when T is above its limit). ctl
+// holds the routing tables and a ticket that is zero at rest.
+struct DecodeBuffers {
+  size_t ctl = 0, dh = 0, hs = 0;
+};
+DecodeBuffers dec_buffers(const v4moe_config& c, int64_t T);
 
 // Workspace carve-up for T tokens. All offsets are 256-byte aligned.
 struct WsLayout {
@@ -39,6 +45,7 @@ struct WsLayout {
   size_t xlog = 0;          // [T, H] f16 activations in the decode layout
   size_t sigma = 0;         // [T] int32 per-token power-of-two exponents
   size_t tc = 0;            // tensor-core path: activations in slot order + tile lists
+  size_t d_ctl = 0, d_dh = 0, d_hs = 0;  // decode path
   size_t total = 0;
   int nchunks = 0;
 };
@@ -65,6 +72,10 @@ inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
   L.xlog = take(size_t(T) * c.hidden * 2);
   L.sigma = take(size_t(T) * 4);
   L.tc = take(tc_extra_bytes(c, T));
+  const DecodeBuffers d = dec_buffers(c, T);
+  L.d_ctl = take(d.ctl);
+  L.d_dh = take(d.dh);
+  L.d_hs = take(d.hs);
   L.total = off;
   return L;
 }
@@ -105,17 +116,35 @@ cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t st);
 // Tensor-core path (tcgen05 grouped GEMMs) for larger token counts.
 cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, cudaStream_t st);
 
-// Decode path (tensor-core weight streaming) for small token counts.
+// Decode path: the whole layer (routing included in layer mode) as three
+// kernels chained by programmatic dependent launch, for at most
+// kDecodeMaxTokens tokens.
 constexpr int kDecodeMaxTokens = 8;
+struct DecodeArgs {
+  v4moe_config c;
+  int T;
+  int layer_mode;  // 1: route in the kernel; 0: topk ids / weights given
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* gate;
+  const float* bias;
+  const int32_t* token_ids;
+  const int32_t* tid2eid;
+  int32_t* topk_ids;
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_slot;
+  int32_t* slot_pos;
+  float* scores;
+  v4moe_weights w;
+  __nv_bfloat16* out;
+  uint32_t* status;
+  uint32_t* ctl;
+  __half* dh;
+  __half* hs;
+};
 bool dec_supported(const v4moe_config& c, int T);
-cudaError_t launch_forward_dec(const ForwardArgs& a, const __half* xlog, const int* sigma, cudaStream_t st);
-cudaError_t launch_dec_xlog(const v4moe_config& c, int T, const __nv_bfloat16* x, __half* xlog, int* sigma,
-                            cudaStream_t st);
-cudaError_t launch_dec_prep(const v4moe_config& c, int T, const __nv_bfloat16* x, const __nv_bfloat16* gate,
-                            const float* bias, const int32_t* token_ids, const int32_t* tid2eid,
-                            int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets,
-                            int32_t* sorted_slot, int32_t* slot_pos, float* scores, __half* xlog, int* sigma,
-                            uint32_t* status, unsigned* ticket, cudaStream_t st);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- device helpers
 

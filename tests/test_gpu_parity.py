@@ -68,6 +68,21 @@ def run_parity(li, layer, n_float_tokens=None, report=None):
     e2e = toks[ok[toks]]
     if e2e.size:
         assert_close(got2[e2e], ref[ok[toks]], f"{wl.name} end-to-end")
+    # routing outputs of the whole-layer call (small batches route inside the
+    # fused decode kernel): ids / weights as the oracle's, permutation exact
+    import mxfp4_routed_expert_v4moe_b200 as V
+    assert V.v4moe_read_device_status(layer.workspace(T)) == V.V4MOE_OK
+    b = layer.buffers(T)
+    ids_l = b["topk_ids"].cpu().numpy()
+    w_l = b["topk_w"].cpu().numpy().astype(np.float64)
+    assert np.array_equal(ids_l[ok], ids_o[ok]), "whole-layer ids differ on non-tie tokens"
+    if ok.any():
+        assert_close(w_l[ok], w_o[ok], "whole-layer topk_w")
+    c_l, off_l, ss_l, sp_l = O.permute(ids_l, wl.E)
+    assert np.array_equal(b["counts"].cpu().numpy(), c_l)
+    assert np.array_equal(b["offsets"].cpu().numpy(), off_l)
+    assert np.array_equal(b["sorted_slot"].cpu().numpy()[:S], ss_l)
+    assert np.array_equal(b["slot_pos"].cpu().numpy()[:S], sp_l)
     if report is not None:
         report.update(near_ties=int(near.sum()), rel_l2=rel, max_abs=mabs, tokens=len(toks))
     return got, ref
