@@ -30,9 +30,10 @@
 //    tokens as the 8 columns) and posts its partial tile to shared memory; the
 //    last warp to post sums the partials in warp order, refills the stage and
 //    writes h as f16 (routed: w * h).
-//  * k_dec_w2: one CTA per SM, sixteen warps owning K blocks i, i + 16, ....
-//    CTA b owns the 16-row output blocks b, b + G, ... and goes through the
-//    shared expert and every routed expert for each of them; a stage holds
+//  * k_dec_w2: two groups of eight warps, warp i of a group owning K blocks
+//    i, i + 8. CTA b owns a run of 16-row output blocks and goes through the
+//    shared expert and every routed expert for each of them, the two groups
+//    taking alternate experts; a stage holds
 //    the expert's 16 weight rows and the intermediates of its tokens. The sum
 //    over experts (shared first, then ascending id) is formed in registers and
 //    written once as bf16, so the result does not depend on timing.
@@ -66,17 +67,14 @@ constexpr int kNJ = 4;             // K blocks per warp held in registers (K <= 
 constexpr int kMaxHit = 64;        // distinct routed experts of a batch (T * k <= 64)
 constexpr uint32_t kBarTries = 1u << 20;
 
-// Control block words (workspace): the ticket is zero at rest; the tables are
-// rewritten by every routing.
+// Control block words (workspace): the routing tables, rewritten by every
+// call for the w2 kernel.
 enum Ctl : int {
-  cTicket = 0,
-  cEpoch = 16,        // calls so far; scores are tagged with epoch + 1
-  cNh = 32,
-  cHit = 64,          // [kMaxHit] expert id per list index
+  cNh = 0,
+  cHit = 32,          // [kMaxHit] expert id per list index
   cMask = cHit + 64,  // [kMaxHit] bit per token routed to the expert
   cW = cMask + 64,    // [kMaxHit][8] float weight per (expert, token)
-  cScores = 1024,     // [8][1024] u64: (tag << 32) | score bits, 8-byte aligned
-  cWords = cScores + 2 * 8 * 1024,
+  cWords = cW + 64 * 8,
 };
 
 struct DecParams {
@@ -245,28 +243,25 @@ __device__ __forceinline__ void tile_s8(const char* ra, const char* rb, bool val
   }
 }
 
-// ---------------------------------------------------------------- routing kernel
+// ---------------------------------------------------------------- routing
 
+// Selection and routing tables, built in shared memory by every w13 CTA.
 struct RouteSmem {
-  int is_last;
   uint32_t bits[32];
   int rank_base[32];
   int cnt[kMaxHit];
   int cum[kMaxHit + 1];
-  int hit[kMaxHit];
-  uint32_t mask[kMaxHit];
-  float wtab[kMaxHit * 8];
   int ids[64];
   float wts[64];
-  int32_t sel_ids[64];  // the selection's output, before it goes to global memory
+  int32_t sel_ids[64];  // the selection's output
   float sel_w[64];
 };
 
-// Publishes the batch's routed experts (ascending ids), per (expert, token)
-// weights and token masks from topk ids / weights (global or shared memory);
-// one warp. Out-of-range ids are skipped and flagged. Returns the expert
-// count.
-__device__ int build_route_meta(RouteSmem& S, const DecParams& P, const int32_t* tids, const float* tw) {
+// The batch's routed experts in ascending id, per (expert, token) weights and
+// token masks, from topk ids / weights (global or shared memory), into tb;
+// one warp. Out-of-range ids are skipped and, unless `quiet`, flagged.
+__device__ __noinline__ void route_tables(RouteSmem& S, Tables& tb, const DecParams& P, const int32_t* tids, const float* tw,
+                             bool quiet) {
   const int lane = threadIdx.x & 31;
   const int Sn = P.T * P.k;
   S.bits[lane] = 0u;
@@ -287,7 +282,7 @@ __device__ int build_route_meta(RouteSmem& S, const DecParams& P, const int32_t*
     S.wts[s] = w;
     if (e >= 0) atomicOr(&S.bits[e >> 5], 1u << (e & 31));
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(P.status, kStatusBadExpertId);
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && !quiet) atomicOr(P.status, kStatusBadExpertId);
   __syncwarp();
   const uint32_t word = S.bits[lane];
   const int c = __popc(word);
@@ -299,9 +294,9 @@ __device__ int build_route_meta(RouteSmem& S, const DecParams& P, const int32_t*
   }
   S.rank_base[lane] = incl - c;
   const int nh = __shfl_sync(0xffffffffu, incl, 31);
-  for (int i = lane; i < kMaxHit * 8; i += 32) S.wtab[i] = 0.f;
+  for (int i = lane; i < kMaxHit * 8; i += 32) tb.w[i] = 0.f;
   for (int i = lane; i < kMaxHit; i += 32) {
-    S.mask[i] = 0u;
+    tb.mask[i] = 0u;
     S.cnt[i] = 0;
   }
   __syncwarp();
@@ -310,26 +305,30 @@ __device__ int build_route_meta(RouteSmem& S, const DecParams& P, const int32_t*
     if (e >= 0) {
       const int r = S.rank_base[e >> 5] + __popc(S.bits[e >> 5] & ((1u << (e & 31)) - 1u));
       const int tok = s / P.k;
-      S.hit[r] = e;
-      atomicAdd(&S.wtab[r * 8 + tok], S.wts[s]);
-      atomicOr(&S.mask[r], 1u << tok);
+      tb.hit[r] = e;
+      atomicAdd(&tb.w[r * 8 + tok], S.wts[s]);
+      atomicOr(&tb.mask[r], 1u << tok);
       atomicAdd(&S.cnt[r], 1);
     }
   }
+  if (lane == 0) tb.nh = nh;
   __syncwarp();
-  float* wg = reinterpret_cast<float*>(P.ctl + cW);
-  for (int i = lane; i < nh; i += 32) {
-    P.ctl[cHit + i] = uint32_t(S.hit[i]);
-    P.ctl[cMask + i] = S.mask[i];
+}
+
+// The tables, for the w2 kernel (one warp).
+__device__ __noinline__ void publish_tables(const Tables& tb, const DecParams& P) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < tb.nh; i += 32) {
+    P.ctl[cHit + i] = uint32_t(tb.hit[i]);
+    P.ctl[cMask + i] = tb.mask[i];
   }
-  for (int i = lane; i < nh * 8; i += 32) wg[i] = S.wtab[i];
-  if (lane == 0) P.ctl[cNh] = uint32_t(nh);
-  return nh;
+  for (int i = lane; i < tb.nh * 8; i += 32) reinterpret_cast<float*>(P.ctl + cW)[i] = tb.w[i];
+  if (lane == 0) P.ctl[cNh] = uint32_t(tb.nh);
 }
 
 // Stable counting sort of the batch's slots by expert (layer-mode outputs),
-// from the tables build_route_meta left in shared memory; one warp.
-__device__ void write_permutation(RouteSmem& S, const DecParams& P, int nh) {
+// from the state route_tables left in shared memory; one warp.
+__device__ __noinline__ void write_permutation(RouteSmem& S, const DecParams& P, int nh) {
   const int lane = threadIdx.x & 31;
   const int Sn = P.T * P.k;
   const int c0 = 2 * lane < nh ? S.cnt[2 * lane] : 0;
@@ -366,35 +365,40 @@ __device__ void write_permutation(RouteSmem& S, const DecParams& P, int nh) {
   }
 }
 
-constexpr int kRouteWarps = 8;
-constexpr uint32_t kSpinTries = 1u << 20;
-
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
-  uint64_t v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
+// Top-k selection of token t (one warp) from scores and bias in shared memory,
+// into the RouteSmem selection arrays. Out of line: the w13 kernel calls it
+// with its activation fragments live.
+template <int NPER>
+__device__ __noinline__ void select_learned_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
+                                                  const float* sbias) {
+  select_learned_n<false, NPER>(t, P.E, P.k, P.routed_scale, ssc + size_t(t) * P.E, sbias, S.sel_ids, S.sel_w);
+}
+__device__ __noinline__ void select_hash_token(RouteSmem& S, const DecParams& P, int t, const float* ssc) {
+  select_hash_warp<true>(t, P.E, P.k, P.vocab, P.routed_scale, ssc + size_t(t) * P.E, P.token_ids, P.tid2eid,
+                         S.sel_ids, S.sel_w, P.status);
+}
+__device__ __forceinline__ void select_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
+                                             const float* sbias) {
+  if (P.token_ids)
+    select_hash_token(S, P, t, ssc);
+  else if (P.E <= 256)
+    select_learned_token<8>(S, P, t, ssc, sbias);
+  else
+    select_learned_token<32>(S, P, t, ssc, sbias);
 }
 
-// Router scores, one warp per expert, then the last CTA selects. The CTAs do
-// not fence: every score carries the call's tag, and the selecting CTA reads
-// each score until the tag is current. Dynamic shared memory: x rows [T][H]
-// bf16, then the scores [T][E] and the bias [E] (fp32) for the selection.
+constexpr int kRouteWarps = 8;
+
+// Router scores s[t, e] (one warp per expert, the x rows staged in shared
+// memory). The selection happens in every CTA of the next kernel.
 __global__ void __launch_bounds__(kRouteWarps * 32) k_dec_route(DecParams P) {
   extern __shared__ __align__(16) char rsm[];
-  __shared__ RouteSmem S;
-  __shared__ uint32_t tag_s;
   // The w13 kernel may start now: before it waits for this grid it only reads
   // the activations and asks L2 for weights.
   pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (!P.layer_mode) {
-    if (warp == 0) build_route_meta(S, P, P.topk_ids, P.topk_w);
-    return;
-  }
   const int H = P.H, T = P.T, E = P.E;
   uint4* xs = reinterpret_cast<uint4*>(rsm);
-  float* ssc = reinterpret_cast<float*>(rsm + size_t(T) * H * 2);
-  float* sbias = ssc + size_t(T) * E;
   const int e = blockIdx.x * kRouteWarps + warp;
   // the whole gate row in flight at once (H <= 4096: up to 16 pieces per lane)
   const uint4* grow = reinterpret_cast<const uint4*>(P.gate + size_t(e < E ? e : 0) * H);
@@ -402,74 +406,28 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_dec_route(DecParams P) {
   uint4 gv[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) gv[i] = i < np ? __ldg(grow + lane + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
-  if (threadIdx.x == 0) tag_s = P.ctl[cEpoch] + 1u;
   for (int i = threadIdx.x; i < T * H / 8; i += blockDim.x) xs[i] = __ldg(reinterpret_cast<const uint4*>(P.x) + i);
   __syncthreads();
-  const uint32_t tag = tag_s;
-  uint64_t* stag = reinterpret_cast<uint64_t*>(P.ctl + cScores);
-  if (e < E)
-    for (int t = 0; t < T; ++t) {
-      const uint4* xrow = xs + size_t(t) * (H / 8);
-      float acc = 0.f;
+  if (e >= E) return;
+  for (int t = 0; t < T; ++t) {
+    const uint4* xrow = xs + size_t(t) * (H / 8);
+    float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (i < np) {
-          const uint4 xv = xrow[lane + 32 * i];
-          acc = fmaf(bf16_lo(gv[i].x), bf16_lo(xv.x), acc);
-          acc = fmaf(bf16_hi(gv[i].x), bf16_hi(xv.x), acc);
-          acc = fmaf(bf16_lo(gv[i].y), bf16_lo(xv.y), acc);
-          acc = fmaf(bf16_hi(gv[i].y), bf16_hi(xv.y), acc);
-          acc = fmaf(bf16_lo(gv[i].z), bf16_lo(xv.z), acc);
-          acc = fmaf(bf16_hi(gv[i].z), bf16_hi(xv.z), acc);
-          acc = fmaf(bf16_lo(gv[i].w), bf16_lo(xv.w), acc);
-          acc = fmaf(bf16_hi(gv[i].w), bf16_hi(xv.w), acc);
-        }
+    for (int i = 0; i < 16; ++i)
+      if (i < np) {
+        const uint4 xv = xrow[lane + 32 * i];
+        acc = fmaf(bf16_lo(gv[i].x), bf16_lo(xv.x), acc);
+        acc = fmaf(bf16_hi(gv[i].x), bf16_hi(xv.x), acc);
+        acc = fmaf(bf16_lo(gv[i].y), bf16_lo(xv.y), acc);
+        acc = fmaf(bf16_hi(gv[i].y), bf16_hi(xv.y), acc);
+        acc = fmaf(bf16_lo(gv[i].z), bf16_lo(xv.z), acc);
+        acc = fmaf(bf16_hi(gv[i].z), bf16_hi(xv.z), acc);
+        acc = fmaf(bf16_lo(gv[i].w), bf16_lo(xv.w), acc);
+        acc = fmaf(bf16_hi(gv[i].w), bf16_hi(xv.w), acc);
+      }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) stag[size_t(t) * 1024 + e] = (uint64_t(tag) << 32) | __float_as_uint(sqrt_softplus_f(acc));
-    }
-  __syncthreads();
-  if (threadIdx.x == 0) S.is_last = atomicAdd(P.ctl + cTicket, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!S.is_last) return;
-  // ---- the selecting CTA: every score of this call, then the selection
-  bool ok = true;
-  for (int i = threadIdx.x; i < T * E; i += blockDim.x) {
-    const int t = i / E, ee = i % E;
-    const uint64_t* src = stag + size_t(t) * 1024 + ee;
-    uint64_t v = ld_relaxed_u64(src);
-    for (uint32_t k = 0; uint32_t(v >> 32) != tag && k < kSpinTries; ++k) {
-      __nanosleep(32);
-      v = ld_relaxed_u64(src);
-    }
-    ok = ok && uint32_t(v >> 32) == tag;
-    ssc[i] = __uint_as_float(uint32_t(v));
-  }
-  if (!ok) atomicOr(P.status, kStatusTimeout);
-  if (!P.token_ids)
-    for (int i = threadIdx.x; i < E; i += blockDim.x) sbias[i] = __ldg(P.bias + i);
-  __syncthreads();
-  if (warp < T) {
-    if (P.token_ids)
-      select_hash_warp<true>(warp, E, P.k, P.vocab, P.routed_scale, ssc + size_t(warp) * E, P.token_ids, P.tid2eid,
-                             S.sel_ids, S.sel_w, P.status);
-    else if (E <= 256)
-      select_learned_n<false, 8>(warp, E, P.k, P.routed_scale, ssc + size_t(warp) * E, sbias, S.sel_ids, S.sel_w);
-    else
-      select_learned_n<false, 32>(warp, E, P.k, P.routed_scale, ssc + size_t(warp) * E, sbias, S.sel_ids, S.sel_w);
-  }
-  __syncthreads();
-  if (warp == 1)
-    for (int i = lane; i < T * P.k; i += 32) {
-      P.topk_ids[i] = S.sel_ids[i];
-      P.topk_w[i] = S.sel_w[i];
-    }
-  if (warp == 0) {
-    write_permutation(S, P, build_route_meta(S, P, S.sel_ids, S.sel_w));
-    if (lane == 0) {
-      P.ctl[cTicket] = 0u;
-      P.ctl[cEpoch] = tag;
-    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) P.scores[size_t(t) * E + e] = sqrt_softplus_f(acc);
   }
 }
 
@@ -482,6 +440,7 @@ struct W13Smem {
   int sigma[8];
   uint32_t xmax[2][kGW][8];
   Tables tb;
+  RouteSmem rt;
 };
 
 constexpr size_t kHead13 = (sizeof(W13Smem) + 127) / 128 * 128;
@@ -670,10 +629,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
       }
   }
 
-  // ---- the routing (previous grid) is complete and visible past this point
+  // ---- routing: every CTA selects from the scores and builds the tables. The
+  // scores and the bias are staged in the (still empty) ring.
+  float* ssc = reinterpret_cast<float*>(stages);
+  float* sbias = ssc + size_t(T) * P.E;
+  if (P.layer_mode && !P.token_ids) {
+    // Run the selection once on whatever the ring holds, results discarded:
+    // its code is then cached when the scores arrive.
+    if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
+    __syncthreads();
+    if (warp == 0) route_tables(S.rt, S.tb, P, S.rt.sel_ids, S.rt.sel_w, true);
+  }
+  // the scores (previous grid) are complete and visible past this point
   pdl_wait();
-  read_tables(S.tb, P);
+  if (P.layer_mode) {
+    for (int i = threadIdx.x; i < T * P.E; i += blockDim.x) ssc[i] = __ldcg(P.scores + i);
+    if (!P.token_ids)
+      for (int i = threadIdx.x; i < P.E; i += blockDim.x) sbias[i] = __ldg(P.bias + i);
+    __syncthreads();
+    if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
+    __syncthreads();
+    if (warp == 0) route_tables(S.rt, S.tb, P, S.rt.sel_ids, S.rt.sel_w, true);
+  } else if (warp == 0) {
+    route_tables(S.rt, S.tb, P, P.topk_ids, P.topk_w, b != 0);
+  }
   __syncthreads();
+  if (b == 0) {  // one CTA writes the routing outputs and the w2 kernel's tables
+    if (warp == 0) publish_tables(S.tb, P);
+    if (P.layer_mode && warp == 1)
+      for (int i = lane; i < T * P.k; i += 32) {
+        P.topk_ids[i] = S.rt.sel_ids[i];
+        P.topk_w[i] = S.rt.sel_w[i];
+      }
+    if (P.layer_mode && warp == 2) write_permutation(S.rt, P, S.tb.nh);
+  }
   const Chunk ch = w13_chunk(P, S.tb.nh, b, G);
   const int npos = ch.size();
   // The routed slabs stream through the ring; the routed w2 rows of this CTA's
@@ -867,26 +856,33 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
     mbar_arrive(&S.full[0]);
   }
 
+  // Two groups of eight warps take alternate expert slots of each output
+  // block; warp i of a group owns K blocks i, i + 8. Every warp keeps its
+  // partial sums over the block's experts in registers; at the end of the
+  // block all sixteen are summed in warp order.
+  const int q = warp >> 3, wi = warp & 7;
   bool ok = true;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int pos = 0; pos < n_items; ++pos) {
-    const Item2 m = w2_item(P, nl, b, pos);
-    const int s = pos % NS;
-    // A timed-out warp keeps going (without reading the stage) so that every
-    // warp reaches the block-end barriers.
-    ok = ok && __all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / NS) & 1u, P));
-    const char* st = stages + size_t(s) * P.stage_bytes;
-    const bool sh = m.li < 0;
-    const int K = sh ? P.Is : P.I;
-    const int nkb = K / 128;
-    if (ok) {
+  for (int r = 0; r < nrb_mine; ++r) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int l = q; l < nl; l += 2) {
+      const int pos = r * nl + l;
+      const Item2 m = w2_item(P, nl, b, pos);
+      const int s = pos % NS;
+      // A timed-out warp keeps going (without reading the stage) so that every
+      // warp reaches the block-end barriers.
+      ok = ok && __all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / NS) & 1u, P));
+      if (!ok) continue;
+      const char* st = stages + size_t(s) * P.stage_bytes;
+      const bool sh = m.li < 0;
+      const int K = sh ? P.Is : P.I;
+      const int nkb = K / 128;
       // B: the intermediates of token g (zero for tokens not routed here)
       const uint32_t mask = sh ? (1u << T) - 1u : S.tb.mask[m.li];
       const bool has_tok = g < T && ((mask >> g) & 1u);
       uint32_t Bf[2][16];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const int kb = warp + 16 * j;
+        const int kb = wi + 8 * j;
         if (has_tok && kb < nkb) {
           const uint4* p4 = reinterpret_cast<const uint4*>(st + w2_hoff(P) + g * K * 2 + kb * 256 + 64 * t);
 #pragma unroll
@@ -904,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
       }
       float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
       if (sh) {
-        tile_s8<2, 16>(st + g * P.Is, st + (g + 8) * P.Is, true, 0, nkb, warp, Bf, a0, a1);
+        tile_s8<2, 8>(st + g * P.Is, st + (g + 8) * P.Is, true, 0, nkb, wi, Bf, a0, a1);
         const float sa = __ldg(P.sh2_scale + m.rb * 16 + g), sb = __ldg(P.sh2_scale + m.rb * 16 + g + 8);
         acc.x += (a0[0] + a1[0]) * sa;
         acc.y += (a0[1] + a1[1]) * sa;
@@ -914,19 +910,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
         const int rs = P.I / 2, Gs = P.I / 32;
         const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + 16 * rs);
         float fa, fb;
-        tile_mx<2, 16>(st + g * rs, st + (g + 8) * rs, sc + g * Gs, sc + (g + 8) * Gs, warp, nkb, Bf, a0, a1, fa,
-                       fb);
+        tile_mx<2, 8>(st + g * rs, st + (g + 8) * rs, sc + g * Gs, sc + (g + 8) * Gs, wi, nkb, Bf, a0, a1, fa, fb);
         acc.x += (a0[0] + a1[0]) * fa;
         acc.y += (a0[1] + a1[1]) * fa;
         acc.z += (a0[2] + a1[2]) * fb;
         acc.w += (a0[3] + a1[3]) * fb;
       }
-      // the last warp to finish with the stage refills it
+      // the last warp of the group to finish with the stage refills it
       __syncwarp();
       int old = 0;
       if (lane == 0) old = atomicAdd(&S.redcnt[s], 1);
       old = __shfl_sync(0xffffffffu, old, 0);
-      if (old == 15) {
+      if (old == 7) {
         if (lane == 0) S.redcnt[s] = 0;
         __syncwarp();
         const int np = pos + NS;
@@ -941,35 +936,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
         }
       }
     }
-    if (m.l == nl - 1) {
-      // block done: sum the 16 warps' partials in warp order, write bf16
-      red[warp * 32 + lane] = acc;
-      __syncthreads();
-      if (warp == 0) {
-        float4 d = red[lane];
-        for (int w = 1; w < 16; ++w) {
-          const float4 v = red[w * 32 + lane];
-          d.x += v.x;
-          d.y += v.y;
-          d.z += v.z;
-          d.w += v.w;
-        }
-        const float v[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int tok = 2 * t + (i & 1);
-          if (tok < T) P.out[size_t(tok) * P.H + m.rb * 16 + g + 8 * (i >> 1)] = __float2bfloat16_rn(v[i]);
-        }
+    // block done: sum the 16 warps' partials in warp order, write bf16
+    red[warp * 32 + lane] = acc;
+    __syncthreads();
+    if (warp == 0) {
+      float4 d = red[lane];
+      for (int w = 1; w < 16; ++w) {
+        const float4 v = red[w * 32 + lane];
+        d.x += v.x;
+        d.y += v.y;
+        d.z += v.z;
+        d.w += v.w;
       }
-      __syncthreads();
-      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float v[4] = {d.x, d.y, d.z, d.w};
+      const int rb = b * P.w2_per + r;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tok = 2 * t + (i & 1);
+        if (tok < T) P.out[size_t(tok) * P.H + rb * 16 + g + 8 * (i >> 1)] = __float2bfloat16_rn(v[i]);
+      }
     }
-  }
-  if (nl == 0) {  // nothing contributes: the output is zero
-    for (int i = threadIdx.x; i < nrb_mine * 16 * T; i += blockDim.x) {
-      const int r = i / (16 * T), rem = i % (16 * T);
-      P.out[size_t(rem / 16) * P.H + (b * P.w2_per + r) * 16 + rem % 16] = __float2bfloat16_rn(0.f);
-    }
+    __syncthreads();
   }
   // No copy may still be landing in this CTA's shared memory.
   __syncthreads();
@@ -990,7 +977,7 @@ Plan make_plan(const v4moe_config& c, int T) {
   Plan p;
   if (T < 1 || T > kDecodeMaxTokens || T * c.top_k > kMaxHit) return p;
   const int H = c.hidden, I = c.inter, Is = c.shared_inter;
-  if (H > kNJ * 8 * 128 || I > 2 * 16 * 128 || Is > 2 * 16 * 128) return p;
+  if (H > kNJ * 8 * 128 || I > 2 * 8 * 128 || Is > 2 * 8 * 128) return p;
   int s13 = 16 * (H / 2) + 16 * (H / 32);
   if (Is > 0) s13 = std::max(s13, 8 * H);
   p.stage13 = (s13 + 127) / 128 * 128;
@@ -1001,7 +988,9 @@ Plan make_plan(const v4moe_config& c, int T) {
   const size_t room = 227 * 1024 - kHead2 - kRed2;
   p.nst2 = int(std::min<size_t>(kMaxStages2, room / p.stage2));
   p.smem2 = kHead2 + size_t(p.nst2) * p.stage2 + kRed2;
-  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2;
+  const size_t route_stage = (size_t(T) * c.n_experts + c.n_experts) * 4;  // scores + bias in the ring
+  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 && route_stage <= size_t(kStages13) * p.stage13 &&
+         size_t(T) * H * 2 <= 227 * 1024;
   return p;
 }
 
@@ -1068,16 +1057,19 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const int nrb = c.hidden / 16;
   P.w2_per = (nrb + sms - 1) / sms;
   const int grid2 = (nrb + P.w2_per - 1) / P.w2_per;
-  const int route_grid = a.layer_mode ? (c.n_experts + kRouteWarps - 1) / kRouteWarps : 1;
-  const size_t route_smem =
-      a.layer_mode ? size_t(a.T) * c.hidden * 2 + size_t(a.T) * c.n_experts * 4 + size_t(c.n_experts) * 4 : 0;
-  set_smem(k_dec_route, route_smem);
-  cudaError_t e =
-      launch_kernel("dec_route", k_dec_route, dim3(route_grid), dim3(kRouteWarps * 32), route_smem, st, false, P);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (a.layer_mode) {
+    const size_t route_smem = size_t(a.T) * c.hidden * 2;
+    set_smem(k_dec_route, route_smem);
+    e = launch_kernel("dec_route", k_dec_route, dim3((c.n_experts + kRouteWarps - 1) / kRouteWarps),
+                      dim3(kRouteWarps * 32), route_smem, st, false, P);
+    if (e != cudaSuccess) return e;
+  }
+  // Without a routing kernel in front, the w13 kernel must not overlap the
+  // previous call's w2 kernel (it rewrites the intermediates that one reads).
   P.stage_bytes = p.stage13;
   set_smem(k_dec_w13, p.smem13);
-  e = launch_kernel("dec_w13", k_dec_w13, dim3(sms), dim3(kThreads), p.smem13, st, true, P);
+  e = launch_kernel("dec_w13", k_dec_w13, dim3(sms), dim3(kThreads), p.smem13, st, a.layer_mode != 0, P);
   if (e != cudaSuccess) return e;
   P.stage_bytes = p.stage2;
   P.nstages = p.nst2;

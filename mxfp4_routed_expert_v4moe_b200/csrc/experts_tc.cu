@@ -73,6 +73,7 @@ struct TcParams {
   int T, H, I, Is, E, k;
   float limit;
   int mode;
+  int tail_tiles;                   // > 0: only the last tail_tiles tiles of the list (the shared expert's)
   const int32_t* offsets;
   const int32_t* sorted_slot;
   const int* sigma;                 // [T] token exponents of the f16 activations
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = B.tmem_base;
   pdl_wait();  // tiles, routing and activations come from earlier kernels
   const int ntiles = *P.ntiles;
+  const int tile0 = P.tail_tiles > 0 ? max(0, ntiles - P.tail_tiles) : 0;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmC_s);
     uint32_t gc = 0;  // global chunk counter
     bool ok = true;
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
+    for (int ti = tile0 + int(blockIdx.x); ti < ntiles && ok; ti += gridDim.x) {
       const TcTile t = P.tiles[ti];
       const TileGeo g = geo(P, t);
       const void* tmB = g.shared ? static_cast<const void*>(&tmB_s) : static_cast<const void*>(&tmB_r);
@@ -271,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     uint32_t gc = 0, lt = 0;
     bool ok = true;
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x, ++lt) {
+    for (int ti = tile0 + int(blockIdx.x); ti < ntiles && ok; ti += gridDim.x, ++lt) {
       const TcTile t = P.tiles[ti];
       const TileGeo g = geo(P, t);
       const uint32_t b = lt & 1u, v = lt >> 1;
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hf = dq & 1;   // half of the 64-element chunk: elements [32 hf, 32 hf + 32)
     uint32_t gc = 0;
     bool ok = true;
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
+    for (int ti = tile0 + int(blockIdx.x); ti < ntiles && ok; ti += gridDim.x) {
       const TcTile t = P.tiles[ti];
       const TileGeo g = geo(P, t);
       int xmax = 0;
@@ -386,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* xch = reinterpret_cast<float*>(smem + kOffX);
     float* inv = reinterpret_cast<float*>(smem + kOffInv);
     uint32_t lt = 0;
-    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x, ++lt) {
+    for (int ti = tile0 + int(blockIdx.x); ti < ntiles; ti += gridDim.x, ++lt) {
       const TcTile t = P.tiles[ti];
       const TileGeo g = geo(P, t);
       const uint32_t b = lt & 1u, v = lt >> 1;
@@ -615,7 +617,8 @@ size_t tc_extra_bytes(const v4moe_config& c, int64_t T) {
                           (std::max(c.inter, c.shared_inter) / 64);
   const int64_t tiles2 = ((S + BN - 1) / BN + c.n_experts + (T + BN - 1) / BN + 2) * (c.hidden / 128);
   return align_up(size_t(S) * c.hidden * 2) + align_up(size_t(tiles13) * sizeof(TcTile)) +
-         align_up(size_t(tiles2) * sizeof(TcTile)) + 256;
+         align_up(size_t(tiles2) * sizeof(TcTile)) + 256 + 2 * align_up(size_t(S) * (c.hidden / 32)) +
+         2 * align_up(size_t(S) * (c.inter / 32));
 }
 
 cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, cudaStream_t st) {
@@ -632,9 +635,29 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   TcTile* t2 = reinterpret_cast<TcTile*>(p);
   p += align_up(size_t(tiles2) * sizeof(TcTile));
   int* counts = reinterpret_cast<int*>(p);  // [0] = n13, [1] = n2
+  p += 256;
+  // Routed experts on block-scaled MMA when the weights allow it: the
+  // activation planes take the place of the f16 slot copies, the intermediate
+  // planes that of the f16 intermediates.
+  const bool mx = mx_supported(c, a.w);
+  MxBuffers mb;
+  mb.xq_hi = reinterpret_cast<uint8_t*>(xperm);
+  mb.xq_lo = mb.xq_hi + size_t(S) * c.hidden;
+  mb.hq_hi = reinterpret_cast<uint8_t*>(a.h);
+  mb.hq_lo = mb.hq_hi + size_t(S) * c.inter;
+  mb.xs_hi = reinterpret_cast<uint8_t*>(p);
+  p += align_up(size_t(S) * (c.hidden / 32));
+  mb.xs_lo = reinterpret_cast<uint8_t*>(p);
+  p += align_up(size_t(S) * (c.hidden / 32));
+  mb.hs_hi = reinterpret_cast<uint8_t*>(p);
+  p += align_up(size_t(S) * (c.inter / 32));
+  mb.hs_lo = reinterpret_cast<uint8_t*>(p);
+  const int tt_sh = c.shared_inter > 0 ? (T + BN - 1) / BN : 0;
+  const int sh13 = tt_sh * (c.shared_inter / 64), sh2 = tt_sh * (c.hidden / 128);
 
-  cudaError_t e = launch_kernel("tc_gather", k_tc_gather, dim3((T + 7) / 8), dim3(256), 0, st, false, T, c.hidden,
-                                c.n_experts, c.top_k, a.x, a.topk_ids, a.slot_pos, x16, xperm, sigma);
+  cudaError_t e = mx ? launch_mx_gather(a, x16, sigma, mb, st)
+                     : launch_kernel("tc_gather", k_tc_gather, dim3((T + 7) / 8), dim3(256), 0, st, false, T,
+                                     c.hidden, c.n_experts, c.top_k, a.x, a.topk_ids, a.slot_pos, x16, xperm, sigma);
   if (e != cudaSuccess) return e;
   e = launch_kernel("tc_tiles", k_tc_tiles, dim3(1), dim3(1024), 0, st, false, T, c.n_experts, c.hidden, c.inter,
                     c.shared_inter, a.offsets, t13, counts, t2, counts + 1);
@@ -689,6 +712,7 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   P.y_slot = a.y_slot;
   P.ys = a.ys;
 
+  P.tail_tiles = 0;
   P.mode = kW13;
   P.w_codes = a.w.w13_codes;
   P.sh_codes = reinterpret_cast<const uint8_t*>(a.w.sh_w13);
@@ -698,9 +722,16 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   P.ntiles = counts;
   P.w_scales = a.w.w13_scales;
   P.sh_scale = a.w.sh_w13_scale;
-  e = launch_kernel("tc_w13", k_tc_gemm, dim3(sms), dim3(kThreads), kSmemBytes, st, true, P, mB_r13, mB_s13, mC_r13,
-                    mC_s13);
-  if (e != cudaSuccess) return e;
+  if (mx) {
+    e = launch_mx_gemm(a, 0, t13, counts, sh13, mb, st);
+    if (e != cudaSuccess) return e;
+    P.tail_tiles = sh13;
+  }
+  if (!mx || sh13 > 0) {
+    e = launch_kernel("tc_w13", k_tc_gemm, dim3(sms), dim3(kThreads), kSmemBytes, st, true, P, mB_r13, mB_s13,
+                      mC_r13, mC_s13);
+    if (e != cudaSuccess) return e;
+  }
 
   P.mode = kW2;
   P.w_codes = a.w.w2_codes;
@@ -711,9 +742,16 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   P.ntiles = counts + 1;
   P.w_scales = a.w.w2_scales;
   P.sh_scale = a.w.sh_w2_scale;
-  e = launch_kernel("tc_w2", k_tc_gemm, dim3(sms), dim3(kThreads), kSmemBytes, st, true, P, mB_r2, mB_s2, mC_r2,
-                    mC_s2);
-  if (e != cudaSuccess) return e;
+  if (mx) {
+    e = launch_mx_gemm(a, 1, t2, counts + 1, sh2, mb, st);
+    if (e != cudaSuccess) return e;
+    P.tail_tiles = sh2;
+  }
+  if (!mx || sh2 > 0) {
+    e = launch_kernel("tc_w2", k_tc_gemm, dim3(sms), dim3(kThreads), kSmemBytes, st, true, P, mB_r2, mB_s2, mC_r2,
+                      mC_s2);
+    if (e != cudaSuccess) return e;
+  }
   return launch_combine(a, st);
 }
 

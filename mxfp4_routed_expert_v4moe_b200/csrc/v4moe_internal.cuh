@@ -113,6 +113,25 @@ struct ForwardArgs {
 
 cudaError_t launch_forward_simt(const ForwardArgs& a, cudaStream_t st);
 cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t st);
+// Routed experts on block-scaled tcgen05 MMA (MXFP4 weights as stored, the
+// activations as two E4M3 planes with E8M0 scales).
+struct MxBuffers {
+  uint8_t* xq_hi;  // [S, H] activation planes in slot order
+  uint8_t* xq_lo;
+  uint8_t* xs_hi;  // [S, H/32] their E8M0 scales
+  uint8_t* xs_lo;
+  uint8_t* hq_hi;  // [S, I] intermediate planes
+  uint8_t* hq_lo;
+  uint8_t* hs_hi;  // [S, I/32]
+  uint8_t* hs_lo;
+};
+bool mx_supported(const v4moe_config& c, const v4moe_weights& w);
+cudaError_t launch_mx_gather(const ForwardArgs& a, __half* x16, int* sigma, const MxBuffers& m, cudaStream_t st);
+// tiles: the tensor-core path's tile list (routed tiles first, shared_tiles
+// trailing ones skipped).
+cudaError_t launch_mx_gemm(const ForwardArgs& a, int w2, const void* tiles, const int* ntiles, int shared_tiles,
+                           const MxBuffers& m, cudaStream_t st);
+
 // Tensor-core path (tcgen05 grouped GEMMs) for larger token counts.
 cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, cudaStream_t st);
 
