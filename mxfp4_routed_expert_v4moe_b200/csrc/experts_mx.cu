@@ -531,6 +531,350 @@ __global__ void __launch_bounds__(kMThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ token-major GEMM
+//
+// For experts with many tokens the roles swap: a tile is 128 slots (MMA M, the
+// activation planes as A) by 256 weight rows (MMA N, the E2M1 codes as B), so
+// one 64 KB stage feeds eight M128 x N256 x K32 MMAs and the weight and
+// activation chunks are each read once per tile. w13 tiles cover 128 channels
+// (their gate rows, then their up rows: accumulator columns 0-127 and
+// 128-255), w2 tiles 256 output rows. The scales also come through TMA, 16
+// bytes (four chunks) per row at a time, into a two-slot ring; the scale
+// warps move them into TMEM. With the operands swapped the epilogue is per
+// thread: lane = slot, so the clamped SwiGLU, the 32-channel block scale and
+// the two h planes need no exchange between threads.
+//
+//   warp 0       TMA producer (operand stages and scale slots)
+//   warp 1       TMEM owner and MMA issuer
+//   warps 2-5    scale writers (TMEM lane quarter = warp % 4)
+//   warps 6-21   epilogue, four per lane quarter, each a quarter of the columns
+constexpr int XM = 128, XN = 256, XK = 128;
+constexpr int kXStages = 3;
+constexpr int kXFirstEpi = 6;
+constexpr int kXEpiWarps = 16;
+constexpr int kXThreads = 32 * (kXFirstEpi + kXEpiWarps);
+constexpr int kXA = XM * XK;            // 16 KB per activation plane
+constexpr int kXB = XN * XK;            // 32 KB: the codes expanded to one byte each
+constexpr int kXStage = 2 * kXA + kXB;  // 64 KB
+constexpr int kXScW = 0;                // scale slot: 256 weight rows, 128 + 128 slot rows, 16 B each
+constexpr int kXScH = XN * 16;
+constexpr int kXScL = kXScH + XM * 16;
+constexpr int kXSc = kXScL + XM * 16;   // 8 KB
+constexpr int kXOffSc = kXStages * kXStage;
+constexpr int kXOffBar = kXOffSc + 2 * kXSc;
+constexpr int kXSmem = kXOffBar + 256 + 1024;
+constexpr uint32_t kXColSF = XN;        // per stage 16 columns: SFA hi (4), SFA lo (4), SFB (8)
+constexpr uint32_t kXTmemCols = 512;
+
+struct XBars {
+  uint64_t full[kXStages];
+  uint64_t empty[kXStages];
+  uint64_t sf_full[kXStages];
+  uint64_t sc_full[2];
+  uint64_t sc_empty[2];
+  uint64_t acc_full, acc_empty, done;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(XBars) <= 256, "barrier block");
+
+struct XGeo {
+  int K, nk;     // reduction length and its chunks of XK
+  int brow0, n;  // first slot and slot count of the tile
+  int wy, wz;    // weight coordinates: w13 (channel, 2 expert), w2 (row, unused)
+};
+
+__device__ __forceinline__ XGeo xgeo(const MxParams& P, const MxTile& t) {
+  XGeo g;
+  g.n = t.n;
+  g.brow0 = P.offsets[t.grp] + t.n0;
+  if (P.mode == kMW13) {
+    g.K = P.H;
+    g.wy = t.row0;
+    g.wz = 2 * t.grp;
+  } else {
+    g.K = P.I;
+    g.wy = t.grp * P.H + t.row0;
+    g.wz = 0;
+  }
+  g.nk = g.K / XK;
+  return g;
+}
+
+// kind::mxf8f6f4 with E4M3 A (activations) and E2M1 B (weights).
+__host__ __device__ constexpr uint32_t idesc_mxt(int M, int N) {
+  return (0u << 7) | (5u << 10) | (uint32_t(N >> 3) << 17) | (1u << 23) | (uint32_t(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kXThreads, 1)
+    k_mxt_gemm(MxParams P, const __grid_constant__ CUtensorMap tmAh, const __grid_constant__ CUtensorMap tmAl,
+               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmSw,
+               const __grid_constant__ CUtensorMap tmSh, const __grid_constant__ CUtensorMap tmSl) {
+  extern __shared__ __align__(1024) char smem_raw[];
+  char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  XBars& B = *reinterpret_cast<XBars*>(smem + kXOffBar);
+  volatile int* abort_flag = &B.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool w13 = P.mode == kMW13;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kXStages; ++s) {
+      mbar_init(&B.full[s], 1);
+      mbar_init(&B.empty[s], 1);
+      mbar_init(&B.sf_full[s], 4);  // one arrival per scale warp
+    }
+    for (int j = 0; j < 2; ++j) {
+      mbar_init(&B.sc_full[j], 1);
+      mbar_init(&B.sc_empty[j], 4);
+    }
+    mbar_init(&B.acc_full, 1);
+    mbar_init(&B.acc_empty, kXEpiWarps);
+    mbar_init(&B.done, 1);
+    B.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&B.tmem_base, kXTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = B.tmem_base;
+  pdl_wait();  // tiles, routing and activations come from earlier kernels
+  const int ntiles = *P.ntiles - P.shared_tiles;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    prefetch_tmap(&tmAh);
+    prefetch_tmap(&tmAl);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSw);
+    prefetch_tmap(&tmSh);
+    prefetch_tmap(&tmSl);
+    uint32_t gc = 0, gs = 0;
+    bool ok = true;
+    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
+      const XGeo g = xgeo(P, P.tiles[ti]);
+      for (int c = 0; c < g.nk; ++c, ++gc) {
+        if ((c & 3) == 0) {  // scales of this chunk and the next three
+          const uint32_t j = gs & 1u, v = gs >> 1;
+          if (!mwait(&B.sc_empty[j], (v & 1u) ^ 1u, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
+          char* sc = smem + kXOffSc + j * kXSc;
+          mbar_arrive_expect_tx(&B.sc_full[j], uint32_t(kXSc));
+          if (w13)
+            tma_load_3d(sc + kXScW, &tmSw, c * 4, g.wy, g.wz, &B.sc_full[j]);
+          else
+            tma_load_2d(sc + kXScW, &tmSw, c * 4, g.wy, &B.sc_full[j]);
+          tma_load_2d(sc + kXScH, &tmSh, c * 4, g.brow0, &B.sc_full[j]);
+          tma_load_2d(sc + kXScL, &tmSl, c * 4, g.brow0, &B.sc_full[j]);
+          ++gs;
+        }
+        const int s = gc % kXStages;
+        const uint32_t u = gc / kXStages;
+        if (!mwait(&B.empty[s], (u & 1u) ^ 1u, abort_flag, P.status)) {
+          ok = false;
+          break;
+        }
+        // E2M1 rows count their packed bytes (64 per row and chunk)
+        mbar_arrive_expect_tx(&B.full[s], uint32_t(2 * kXA + XN * XK / 2));
+        char* st = smem + s * kXStage;
+        tma_load_2d(st, &tmAh, c * XK, g.brow0, &B.full[s]);
+        tma_load_2d(st + kXA, &tmAl, c * XK, g.brow0, &B.full[s]);
+        if (w13)  // gate and up rows of 128 channels in one box of the 3-D map
+          tma_load_3d(st + 2 * kXA, &tmB, c * XK, g.wy, g.wz, &B.full[s]);
+        else
+          tma_load_2d(st + 2 * kXA, &tmB, c * XK, g.wy, &B.full[s]);
+      }
+    }
+    // nothing may still be landing in shared memory when the CTA exits
+    for (uint32_t q = 0; q < uint32_t(kXStages) && q < gc; ++q) {
+      const uint32_t gq = gc - 1 - q;
+      mbar_wait_bounded(&B.full[gq % kXStages], (gq / kXStages) & 1u, kMTries);
+    }
+    for (uint32_t q = 0; q < 2u && q < gs; ++q) {
+      const uint32_t gq = gs - 1 - q;
+      mbar_wait_bounded(&B.sc_full[gq & 1u], (gq >> 1) & 1u, kMTries);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    uint32_t gc = 0, lt = 0;
+    bool ok = true;
+    const uint32_t idesc = idesc_mxt(XM, XN);
+    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x, ++lt) {
+      const XGeo g = xgeo(P, P.tiles[ti]);
+      if (!mwait(&B.acc_empty, (lt & 1u) ^ 1u, abort_flag, P.status)) break;
+      tc_fence_after();
+      for (int c = 0; c < g.nk; ++c, ++gc) {
+        const int s = gc % kXStages;
+        const uint32_t u = gc / kXStages;
+        if (!mwait(&B.full[s], u & 1u, abort_flag, P.status) ||
+            !mwait(&B.sf_full[s], u & 1u, abort_flag, P.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ah = smem_u32(smem + s * kXStage);
+        const uint32_t al = ah + kXA;
+        const uint32_t bw = ah + 2 * kXA;
+        const uint32_t sf = tmem + kXColSF + 16u * uint32_t(s);
+#pragma unroll
+        for (int kk = 0; kk < XK / 32; ++kk) {
+          const uint32_t id = idesc | (uint32_t(kk) << 29) | (uint32_t(kk) << 4);
+          const uint32_t byte = uint32_t(kk) << 30;
+          const uint64_t bd = sw128_kmajor_desc(bw + kk * 32);
+          umma_mx(tmem, sw128_kmajor_desc(ah + kk * 32), bd, id, (c > 0 || kk > 0) ? 1u : 0u, sf | byte,
+                  (sf + 8) | byte);
+          umma_mx(tmem, sw128_kmajor_desc(al + kk * 32), bd, id, 1u, (sf + 4) | byte, (sf + 8) | byte);
+        }
+        umma_commit(&B.empty[s]);
+      }
+      if (!ok) break;
+      umma_commit(&B.acc_full);
+    }
+    umma_commit(&B.done);
+    mbar_wait_bounded(&B.done, 0, kMTries);
+  } else if (warp >= 2 && warp < kXFirstEpi) {
+    // ------------------------------------------------------------ scale writers
+    // Lane l of every lane quarter holds operand row 32 i + l in column i, one
+    // byte per K step: columns 0-3 the slots' hi scales, 4-7 their lo scales,
+    // 8-15 the 256 weight rows.
+    const int q = warp & 3;
+    uint32_t gc = 0, gs = 0;
+    bool ok = true;
+    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
+      const XGeo g = xgeo(P, P.tiles[ti]);
+      for (int c = 0; c < g.nk && ok; ++c, ++gc) {
+        const uint32_t j = gs & 1u;
+        if ((c & 3) == 0 && !__all_sync(0xffffffffu, mwait(&B.sc_full[j], (gs >> 1) & 1u, abort_flag, P.status))) {
+          ok = false;
+          break;
+        }
+        const int s = gc % kXStages;
+        const uint32_t u = gc / kXStages;
+        if (!__all_sync(0xffffffffu, mwait(&B.empty[s], (u & 1u) ^ 1u, abort_flag, P.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const char* sc = smem + kXOffSc + j * kXSc + 4 * (c & 3);
+        uint32_t wv[8], hv[4], lv[4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wv[i] = *reinterpret_cast<const uint32_t*>(sc + kXScW + (32 * i + lane) * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          hv[i] = *reinterpret_cast<const uint32_t*>(sc + kXScH + (32 * i + lane) * 16);
+          lv[i] = *reinterpret_cast<const uint32_t*>(sc + kXScL + (32 * i + lane) * 16);
+        }
+        const uint32_t ta = tmem + kXColSF + 16u * uint32_t(s) + (uint32_t(32 * q) << 16);
+        tmem_st_32x32b_x4(ta, hv[0], hv[1], hv[2], hv[3]);
+        tmem_st_32x32b_x4(ta + 4, lv[0], lv[1], lv[2], lv[3]);
+        tmem_st_32x32b_x8(ta + 8, wv);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&B.sf_full[s]);
+          if ((c & 3) == 3) mbar_arrive(&B.sc_empty[j]);
+        }
+        if ((c & 3) == 3) ++gs;
+      }
+    }
+  } else if (warp >= kXFirstEpi) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                  // TMEM lane quarter
+    const int sub = (warp - kXFirstEpi) >> 2;  // quarter of the columns
+    const int row = 32 * q + lane;
+    uint32_t lt = 0;
+    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x, ++lt) {
+      const MxTile t = P.tiles[ti];
+      const XGeo g = xgeo(P, t);
+      if (!__all_sync(0xffffffffu, mwait(&B.acc_full, lt & 1u, abort_flag, P.status)) || *abort_flag) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t(32 * q) << 16);
+      const bool valid = row < g.n;
+      const size_t slot = size_t(g.brow0 + row);
+      if (w13) {
+        // columns 32 sub .. +31 (gate) and 128 + 32 sub .. (up): one 32-channel block
+        uint32_t gr[32], ur[32];
+        tmem_ld_32x32b_x32(acc + 32 * sub, gr);
+        tmem_ld_32x32b_x32(acc + XN / 2 + 32 * sub, ur);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.acc_empty);
+        if (valid) {
+          uint32_t am = 0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float h = clamped_swiglu_f(__uint_as_float(gr[i]), __uint_as_float(ur[i]), P.limit);
+            gr[i] = __float_as_uint(h);
+            am = max(am, gr[i] & 0x7FFFFFFFu);
+          }
+          const int se = block_exp(am);
+          uint32_t hw[8], lw[8];
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {
+            hw[w] = 0u;
+            lw[w] = 0u;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              uint8_t hb, lb;
+              split_e4m3(__uint_as_float(gr[4 * w + b]), se, hb, lb);
+              hw[w] |= uint32_t(hb) << (8 * b);
+              lw[w] |= uint32_t(lb) << (8 * b);
+            }
+          }
+          const int ch = t.row0 + 32 * sub;
+          uint4* dh = reinterpret_cast<uint4*>(P.h_hi + slot * P.I + ch);
+          uint4* dl = reinterpret_cast<uint4*>(P.h_lo + slot * P.I + ch);
+          dh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          dh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+          dl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          dl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+          P.hs_hi[slot * (P.I / 32) + ch / 32] = uint8_t(se + 127);
+          P.hs_lo[slot * (P.I / 32) + ch / 32] = uint8_t(max(1, se + 123));
+        }
+      } else {
+        // columns 64 sub .. +63 of the 256 output rows
+        uint32_t ya[32], yb[32];
+        tmem_ld_32x32b_x32(acc + 64 * sub, ya);
+        tmem_ld_32x32b_x32(acc + 64 * sub + 32, yb);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.acc_empty);
+        if (valid) {
+          float4* dy = reinterpret_cast<float4*>(P.y_slot + slot * P.H + t.row0 + 64 * sub);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dy[i] = make_float4(__uint_as_float(ya[4 * i]), __uint_as_float(ya[4 * i + 1]),
+                                __uint_as_float(ya[4 * i + 2]), __uint_as_float(ya[4 * i + 3]));
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dy[8 + i] = make_float4(__uint_as_float(yb[4 * i]), __uint_as_float(yb[4 * i + 1]),
+                                    __uint_as_float(yb[4 * i + 2]), __uint_as_float(yb[4 * i + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kXTmemCols);
+  }
+}
+
 
 PFN_cuTensorMapEncodeTiled_v12000 mx_encode_fn() {
   static std::once_flag once;
@@ -572,6 +916,32 @@ bool mx_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t c
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
+}
+
+// General 2-D / 3-D maps ([halves][rows][cols], rows row_bytes apart).
+bool mx_map2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t row_bytes, uint64_t rows,
+              uint32_t bx, uint32_t by, CUtensorMapSwizzle sw) {
+  auto fn = mx_encode_fn();
+  if (!fn) return false;
+  if (rows == 0) rows = 1;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {bx, by};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool mx_map3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t row_bytes, uint64_t rows,
+              uint64_t halves, uint32_t bx, uint32_t by, CUtensorMapSwizzle sw) {
+  auto fn = mx_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {cols, rows, halves};
+  const cuuint64_t strides[2] = {row_bytes, rows * row_bytes};
+  const cuuint32_t box[3] = {bx, by, 2};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -637,6 +1007,62 @@ cudaError_t launch_mx_gemm(const ForwardArgs& a, int w2, const void* tiles, cons
   set_smem(k_mx_gemm, kMSmem);
   return launch_kernel(w2 ? "mx_w2" : "mx_w13", k_mx_gemm, dim3(sms), dim3(kMThreads), kMSmem, st, true, P, mA, mBh,
                        mBl);
+}
+
+cudaError_t launch_mxt_gemm(const ForwardArgs& a, int w2, const void* tiles, const int* ntiles, int shared_tiles,
+                            const MxBuffers& m, cudaStream_t st) {
+  const v4moe_config& c = a.c;
+  const uint64_t S = uint64_t(a.T) * c.top_k;
+  const uint64_t H = c.hidden, I = c.inter, E = c.n_experts;
+  MxParams P;
+  P.T = a.T;
+  P.H = c.hidden;
+  P.I = c.inter;
+  P.E = c.n_experts;
+  P.k = c.top_k;
+  P.limit = c.swiglu_limit;
+  P.mode = w2 ? kMW2 : kMW13;
+  P.offsets = a.offsets;
+  P.tiles = static_cast<const MxTile*>(tiles);
+  P.ntiles = ntiles;
+  P.shared_tiles = shared_tiles;
+  P.h_hi = m.hq_hi;
+  P.h_lo = m.hq_lo;
+  P.hs_hi = m.hs_hi;
+  P.hs_lo = m.hs_lo;
+  P.y_slot = a.y_slot;
+  P.status = a.status;
+  P.w_scales = nullptr;
+  P.b_sc_hi = nullptr;
+  P.b_sc_lo = nullptr;
+  constexpr auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  constexpr auto U4 = CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+  constexpr auto SW = CU_TENSOR_MAP_SWIZZLE_128B;
+  constexpr auto NS = CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUtensorMap mAh, mAl, mB, mSw, mSh, mSl;
+  bool ok = true;
+  if (!w2) {
+    ok &= mx_map2d(&mAh, m.xq_hi, U8, H, H, S, XK, XM, SW);
+    ok &= mx_map2d(&mAl, m.xq_lo, U8, H, H, S, XK, XM, SW);
+    ok &= mx_map3d(&mB, a.w.w13_codes, U4, H, H / 2, I, 2 * E, XK, XN / 2, SW);
+    ok &= mx_map3d(&mSw, a.w.w13_scales, U8, H / 32, H / 32, I, 2 * E, 16, XN / 2, NS);
+    ok &= mx_map2d(&mSh, m.xs_hi, U8, H / 32, H / 32, S, 16, XM, NS);
+    ok &= mx_map2d(&mSl, m.xs_lo, U8, H / 32, H / 32, S, 16, XM, NS);
+  } else {
+    ok &= mx_map2d(&mAh, m.hq_hi, U8, I, I, S, XK, XM, SW);
+    ok &= mx_map2d(&mAl, m.hq_lo, U8, I, I, S, XK, XM, SW);
+    ok &= mx_map2d(&mB, a.w.w2_codes, U4, I, I / 2, E * H, XK, XN, SW);
+    ok &= mx_map2d(&mSw, a.w.w2_scales, U8, I / 32, I / 32, E * H, 16, XN, NS);
+    ok &= mx_map2d(&mSh, m.hs_hi, U8, I / 32, I / 32, S, 16, XM, NS);
+    ok &= mx_map2d(&mSl, m.hs_lo, U8, I / 32, I / 32, S, 16, XM, NS);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  set_smem(k_mxt_gemm, kXSmem);
+  return launch_kernel(w2 ? "mxt_w2" : "mxt_w13", k_mxt_gemm, dim3(sms), dim3(kXThreads), kXSmem, st, true, P, mAh,
+                       mAl, mB, mSw, mSh, mSl);
 }
 
 }  // namespace v4moe

@@ -516,7 +516,8 @@ __global__ void __launch_bounds__(256) k_tc_gather(int T, int H, int E, int k, c
 
 // Tile lists of both GEMMs (one CTA, one group per thread): per group
 // (routed experts in id order, then the shared expert), token tiles of <= BN,
-// times the row blocks (64 channels for w13, 128 output rows for w2). The
+// times the row blocks: for the routed experts rb13 channels (w13) and rb2
+// output rows (w2), for the shared expert 64 channels and 128 rows. The
 // groups' tile counts are prefix-summed across the block.
 __device__ __forceinline__ int block_excl_scan_1024(int v, int* warp_tot, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -543,7 +544,8 @@ __device__ __forceinline__ int block_excl_scan_1024(int v, int* warp_tot, int* t
   return warp_tot[warp] + incl - v;
 }
 
-__global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, int Is, const int32_t* __restrict__ offsets,
+__global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, int Is, int rb13, int rb2,
+                                                   const int32_t* __restrict__ offsets,
                                                    TcTile* __restrict__ t13, int* __restrict__ n13, TcTile* __restrict__ t2,
                                                    int* __restrict__ n2) {
   __shared__ int wt13[32], wt2[32];
@@ -555,8 +557,8 @@ __global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, i
     if (g < G) {
       n[q] = g < E ? offsets[g + 1] - offsets[g] : T;
       const int tt = (n[q] + BN - 1) / BN;
-      c13[q] = tt * ((g < E ? I : Is) / 64);
-      c2[q] = tt * (H / 128);
+      c13[q] = tt * (g < E ? I / rb13 : Is / 64);
+      c2[q] = tt * (g < E ? H / rb2 : H / 128);
     }
   }
   // second group of a thread (only the shared expert when E == 1024) follows all first groups
@@ -571,11 +573,12 @@ __global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, i
     const int g = threadIdx.x + q * 1024;
     if (g >= G || (q == 1 && threadIdx.x != 0)) continue;
     const int tt = (n[q] + BN - 1) / BN;
-    const int nb13 = (g < E ? I : Is) / 64, nb2 = H / 128;
+    const int r13 = g < E ? rb13 : 64, r2 = g < E ? rb2 : 128;
+    const int nb13 = (g < E ? I : Is) / r13, nb2 = H / r2;
     for (int i = 0; i < tt; ++i) {
       const int n0 = i * BN, nn = min(BN, n[q] - n0);
-      for (int bb = 0; bb < nb13; ++bb) t13[base13[q] + i * nb13 + bb] = TcTile{g, bb * 64, n0, nn};
-      for (int bb = 0; bb < nb2; ++bb) t2[base2[q] + i * nb2 + bb] = TcTile{g, bb * 128, n0, nn};
+      for (int bb = 0; bb < nb13; ++bb) t13[base13[q] + i * nb13 + bb] = TcTile{g, bb * r13, n0, nn};
+      for (int bb = 0; bb < nb2; ++bb) t2[base2[q] + i * nb2 + bb] = TcTile{g, bb * r2, n0, nn};
     }
   }
 }
@@ -659,8 +662,11 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
                      : launch_kernel("tc_gather", k_tc_gather, dim3((T + 7) / 8), dim3(256), 0, st, false, T,
                                      c.hidden, c.n_experts, c.top_k, a.x, a.topk_ids, a.slot_pos, x16, xperm, sigma);
   if (e != cudaSuccess) return e;
+  // Token-major block-scaled tiles (128 slots x 256 weight rows) once the
+  // experts average enough tokens to fill them; weight-major ones otherwise.
+  const bool mxt = mx && int64_t(T) * c.top_k >= int64_t(kMxtMinAvg) * c.n_experts;
   e = launch_kernel("tc_tiles", k_tc_tiles, dim3(1), dim3(1024), 0, st, false, T, c.n_experts, c.hidden, c.inter,
-                    c.shared_inter, a.offsets, t13, counts, t2, counts + 1);
+                    c.shared_inter, mxt ? 128 : 64, mxt ? 256 : 128, a.offsets, t13, counts, t2, counts + 1);
   if (e != cudaSuccess) return e;
 
   // tensor maps
@@ -723,7 +729,7 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   P.w_scales = a.w.w13_scales;
   P.sh_scale = a.w.sh_w13_scale;
   if (mx) {
-    e = launch_mx_gemm(a, 0, t13, counts, sh13, mb, st);
+    e = mxt ? launch_mxt_gemm(a, 0, t13, counts, sh13, mb, st) : launch_mx_gemm(a, 0, t13, counts, sh13, mb, st);
     if (e != cudaSuccess) return e;
     P.tail_tiles = sh13;
   }
@@ -743,7 +749,7 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   P.w_scales = a.w.w2_scales;
   P.sh_scale = a.w.sh_w2_scale;
   if (mx) {
-    e = launch_mx_gemm(a, 1, t2, counts + 1, sh2, mb, st);
+    e = mxt ? launch_mxt_gemm(a, 1, t2, counts + 1, sh2, mb, st) : launch_mx_gemm(a, 1, t2, counts + 1, sh2, mb, st);
     if (e != cudaSuccess) return e;
     P.tail_tiles = sh2;
   }

@@ -131,6 +131,11 @@ cudaError_t launch_mx_gather(const ForwardArgs& a, __half* x16, int* sigma, cons
 // trailing ones skipped).
 cudaError_t launch_mx_gemm(const ForwardArgs& a, int w2, const void* tiles, const int* ntiles, int shared_tiles,
                            const MxBuffers& m, cudaStream_t st);
+// Token-major variant (128 slots x 256 weight rows per tile), for experts that
+// average at least kMxtMinAvg tokens.
+constexpr int kMxtMinAvg = 48;
+cudaError_t launch_mxt_gemm(const ForwardArgs& a, int w2, const void* tiles, const int* ntiles, int shared_tiles,
+                            const MxBuffers& m, cudaStream_t st);
 
 // Tensor-core path (tcgen05 grouped GEMMs) for larger token counts.
 cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, cudaStream_t st);
