@@ -77,24 +77,41 @@ def algorithmic(wl, ids, token_ids=None):
         route_b = E * H * 2 + T * 4 + n_tok * k * 4  # gate + token ids + touched table rows
     step_b = n_hit * (e13 + e2) + s13 + s2 + route_b + 4 * T * H + 48 * T
     flops = S * 6 * H * I + T * 6 * H * Is + 2 * T * E * H
+    # per kernel kind: routed experts only, shared expert only, or both in one kernel
+    r13_b = n_hit * e13 + T * H * 2 + S * I * 2
+    r2_b = n_hit * e2 + S * I * 2 + S * H * 4
+    sh13_b = s13 + T * H * 2 + T * Is * 2
+    sh2_b = s2 + T * Is * 2 + S * H * 4 + T * H * 2
+    r13_f, r2_f = S * 2 * (2 * I) * H, S * 2 * H * I
+    sh13_f, sh2_f = T * 2 * (2 * Is) * H, T * 2 * H * Is
     per_kernel_bytes = {
+        "routed_w13": r13_b, "routed_w2": r2_b, "shared_w13": sh13_b, "shared_w2": sh2_b,
         "w13": n_hit * e13 + s13 + T * H * 2 + S * I * 2 + T * Is * 2,
         "w2": n_hit * e2 + s2 + S * I * 2 + T * Is * 2 + T * H * 2,
     }
     per_kernel_flops = {
-        "w13": S * 2 * (2 * I) * H + T * 2 * (2 * Is) * H,
-        "w2": S * 2 * H * I + T * 2 * H * Is,
+        "routed_w13": r13_f, "routed_w2": r2_f, "shared_w13": sh13_f, "shared_w2": sh2_f,
+        "w13": r13_f + sh13_f, "w2": r2_f + sh2_f,
     }
     return dict(n_hit=n_hit, step_bytes=step_b, step_flops=flops, kernel_bytes=per_kernel_bytes,
                 kernel_flops=per_kernel_flops)
 
 
 def kernel_kind(name):
-    if "w13" in name:
-        return "w13"
-    if "w2" in name:
-        return "w2"
-    return None
+    """Which part of the layer a kernel computes: the decode kernels take the
+    routed experts and the shared expert together; on the tensor-core path the
+    block-scaled kernels (mx*, mxt*) take the routed experts and the f16 ones
+    (sh*, tc*) the shared expert."""
+    part = "w13" if "w13" in name else "w2" if "w2" in name else None
+    if part is None:
+        return None
+    if name.startswith("dec_"):
+        return part
+    if name.startswith("mx"):
+        return "routed_" + part
+    if name.startswith(("sh_", "tc_")):
+        return "shared_" + part
+    return part
 
 
 def peaks():

@@ -206,6 +206,8 @@ WORKLOADS = {
     # the weights under 1 GB; per-expert token counts match the full cases).
     "decode_b1_e64": Workload("decode_b1_e64", T=1, E=64,
                               notes="decode batch 1 with 64 experts (profiling size)"),
+    "decode_b64_e64": Workload("decode_b64_e64", T=64, E=64, bias_std=0.5,
+                               notes="decode batch 64 with 64 experts (profiling size)"),
     "prefill_1024_e64": Workload("prefill_1024_e64", T=1024, E=64,
                                  notes="prefill, ~96 tokens per expert, 64 experts (profiling size)"),
 }

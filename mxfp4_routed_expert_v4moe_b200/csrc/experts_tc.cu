@@ -514,11 +514,12 @@ __global__ void __launch_bounds__(256) k_tc_gather(int T, int H, int E, int k, c
   }
 }
 
-// Tile lists of both GEMMs (one CTA, one group per thread): per group
-// (routed experts in id order, then the shared expert), token tiles of <= BN,
-// times the row blocks: for the routed experts rb13 channels (w13) and rb2
-// output rows (w2), for the shared expert 64 channels and 128 rows. The
-// groups' tile counts are prefix-summed across the block.
+// Tile lists of both GEMMs (one CTA): per group (routed experts in id order,
+// then the shared expert unless Is == 0), token tiles of <= BN, times the row
+// blocks: for the routed experts rb13 channels (w13) and rb2 output rows (w2),
+// for the shared expert 64 channels and 128 rows. One thread counts a group's
+// tiles, the counts are prefix-summed across the block, and one warp writes a
+// group's entries.
 __device__ __forceinline__ int block_excl_scan_1024(int v, int* warp_tot, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = v;
@@ -550,35 +551,50 @@ __global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, i
                                                    int* __restrict__ n2) {
   __shared__ int wt13[32], wt2[32];
   __shared__ int tot13, tot2;
+  __shared__ int gn[1025], gb13[1025], gb2[1025];
   const int G = E + (Is > 0 ? 1 : 0);  // <= 1025 groups: threads take g and g + 1024
-  int n[2] = {0, 0}, c13[2] = {0, 0}, c2[2] = {0, 0};
+  int c13[2] = {0, 0}, c2[2] = {0, 0};
   for (int q = 0; q < 2; ++q) {
     const int g = threadIdx.x + q * 1024;
     if (g < G) {
-      n[q] = g < E ? offsets[g + 1] - offsets[g] : T;
-      const int tt = (n[q] + BN - 1) / BN;
+      const int n = g < E ? offsets[g + 1] - offsets[g] : T;
+      const int tt = (n + BN - 1) / BN;
+      gn[g] = n;
       c13[q] = tt * (g < E ? I / rb13 : Is / 64);
       c2[q] = tt * (g < E ? H / rb2 : H / 128);
     }
   }
-  // second group of a thread (only the shared expert when E == 1024) follows all first groups
+  // the second group of a thread (only the shared expert when E == 1024) follows all first groups
   const int b13 = block_excl_scan_1024(c13[0], wt13, &tot13);
   const int b2 = block_excl_scan_1024(c2[0], wt2, &tot2);
-  int base13[2] = {b13, tot13}, base2[2] = {b2, tot2};
+  if (threadIdx.x < G) {
+    gb13[threadIdx.x] = b13;
+    gb2[threadIdx.x] = b2;
+  }
   if (threadIdx.x == 0) {
+    if (G > 1024) {
+      gb13[1024] = tot13;
+      gb2[1024] = tot2;
+    }
     *n13 = tot13 + c13[1];
     *n2 = tot2 + c2[1];
   }
-  for (int q = 0; q < 2; ++q) {
-    const int g = threadIdx.x + q * 1024;
-    if (g >= G || (q == 1 && threadIdx.x != 0)) continue;
-    const int tt = (n[q] + BN - 1) / BN;
+  __syncthreads();
+  // one warp per group, its lanes over the group's tiles (token tile major,
+  // then row block)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int g = warp; g < G; g += 32) {
+    const int n = gn[g];
+    const int tt = (n + BN - 1) / BN;
     const int r13 = g < E ? rb13 : 64, r2 = g < E ? rb2 : 128;
     const int nb13 = (g < E ? I : Is) / r13, nb2 = H / r2;
-    for (int i = 0; i < tt; ++i) {
-      const int n0 = i * BN, nn = min(BN, n[q] - n0);
-      for (int bb = 0; bb < nb13; ++bb) t13[base13[q] + i * nb13 + bb] = TcTile{g, bb * r13, n0, nn};
-      for (int bb = 0; bb < nb2; ++bb) t2[base2[q] + i * nb2 + bb] = TcTile{g, bb * r2, n0, nn};
+    for (int i = lane; i < tt * nb13; i += 32) {
+      const int n0 = (i / nb13) * BN;
+      t13[gb13[g] + i] = TcTile{g, (i % nb13) * r13, n0, min(BN, n - n0)};
+    }
+    for (int i = lane; i < tt * nb2; i += 32) {
+      const int n0 = (i / nb2) * BN;
+      t2[gb2[g] + i] = TcTile{g, (i % nb2) * r2, n0, min(BN, n - n0)};
     }
   }
 }
@@ -624,7 +640,8 @@ size_t tc_extra_bytes(const v4moe_config& c, int64_t T) {
          2 * align_up(size_t(S) * (c.inter / 32));
 }
 
-cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, cudaStream_t st) {
+cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, char* sh16,
+                              cudaStream_t st) {
   const v4moe_config& c = a.c;
   const int T = a.T;
   const int64_t S = int64_t(T) * c.top_k;
@@ -655,7 +672,10 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   mb.hs_hi = reinterpret_cast<uint8_t*>(p);
   p += align_up(size_t(S) * (c.inter / 32));
   mb.hs_lo = reinterpret_cast<uint8_t*>(p);
-  const int tt_sh = c.shared_inter > 0 ? (T + BN - 1) / BN : 0;
+  // Shared expert on its own f16 GEMM (large batches, block-scaled path only);
+  // otherwise its tiles trail the routed ones in the lists.
+  const bool shx = mx && sh_supported(c, T);
+  const int tt_sh = c.shared_inter > 0 && !shx ? (T + BN - 1) / BN : 0;
   const int sh13 = tt_sh * (c.shared_inter / 64), sh2 = tt_sh * (c.hidden / 128);
 
   cudaError_t e = mx ? launch_mx_gather(a, x16, sigma, mb, st)
@@ -666,7 +686,8 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   // experts average enough tokens to fill them; weight-major ones otherwise.
   const bool mxt = mx && int64_t(T) * c.top_k >= int64_t(kMxtMinAvg) * c.n_experts;
   e = launch_kernel("tc_tiles", k_tc_tiles, dim3(1), dim3(1024), 0, st, false, T, c.n_experts, c.hidden, c.inter,
-                    c.shared_inter, mxt ? 128 : 64, mxt ? 256 : 128, a.offsets, t13, counts, t2, counts + 1);
+                    shx ? 0 : c.shared_inter, mxt ? 128 : 64, mxt ? 256 : 128, a.offsets, t13, counts, t2,
+                    counts + 1);
   if (e != cudaSuccess) return e;
 
   // tensor maps
@@ -732,6 +753,7 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
     e = mxt ? launch_mxt_gemm(a, 0, t13, counts, sh13, mb, st) : launch_mx_gemm(a, 0, t13, counts, sh13, mb, st);
     if (e != cudaSuccess) return e;
     P.tail_tiles = sh13;
+    if (shx && (e = launch_sh_w13(a, x16, sigma, sh16, st)) != cudaSuccess) return e;
   }
   if (!mx || sh13 > 0) {
     e = launch_kernel("tc_w13", k_tc_gemm, dim3(sms), dim3(kThreads), kSmemBytes, st, true, P, mB_r13, mB_s13,
@@ -752,6 +774,7 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
     e = mxt ? launch_mxt_gemm(a, 1, t2, counts + 1, sh2, mb, st) : launch_mx_gemm(a, 1, t2, counts + 1, sh2, mb, st);
     if (e != cudaSuccess) return e;
     P.tail_tiles = sh2;
+    if (shx) return launch_sh_w2_combine(a, sh16, st);  // the combine is in its epilogue
   }
   if (!mx || sh2 > 0) {
     e = launch_kernel("tc_w2", k_tc_gemm, dim3(sms), dim3(kThreads), kSmemBytes, st, true, P, mB_r2, mB_s2, mC_r2,

@@ -205,7 +205,8 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x, const i
     return launch_status(launch_decode(d, st));
   }
   const ForwardArgs a = forward_args(cfg, T, x, topk_ids, topk_w, offsets, sorted_slot, slot_pos, weights, out, ws);
-  return launch_status(launch_forward_tc(a, at<__half>(ws, L.xlog), at<int>(ws, L.sigma), at<char>(ws, L.tc), st));
+  return launch_status(
+      launch_forward_tc(a, at<__half>(ws, L.xlog), at<int>(ws, L.sigma), at<char>(ws, L.tc), at<char>(ws, L.sh16), st));
 }
 
 int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const void* gate, const float* bias,

@@ -25,6 +25,11 @@ constexpr int kPermChunk = 2048;
 
 size_t tc_extra_bytes(const v4moe_config& c, int64_t T);
 
+// Shared expert on the token-major f16 GEMM (int8 weights widened to f16 in
+// the workspace) from this many tokens on.
+constexpr int kShMinTokens = 512;
+size_t sh_extra_bytes(const v4moe_config& c, int64_t T);
+
 // Buffers of the decode path (all zero bytes when T is above its limit). ctl
 // holds the routing tables and a ticket that is zero at rest.
 struct DecodeBuffers {
@@ -45,6 +50,7 @@ struct WsLayout {
   size_t xlog = 0;          // [T, H] f16 activations in the decode layout
   size_t sigma = 0;         // [T] int32 per-token power-of-two exponents
   size_t tc = 0;            // tensor-core path: activations in slot order + tile lists
+  size_t sh16 = 0;          // shared expert weights widened to f16 (large batches)
   size_t d_ctl = 0, d_dh = 0, d_hs = 0;  // decode path
   size_t total = 0;
   int nchunks = 0;
@@ -72,6 +78,7 @@ inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
   L.xlog = take(size_t(T) * c.hidden * 2);
   L.sigma = take(size_t(T) * 4);
   L.tc = take(tc_extra_bytes(c, T));
+  L.sh16 = take(sh_extra_bytes(c, T));
   const DecodeBuffers d = dec_buffers(c, T);
   L.d_ctl = take(d.ctl);
   L.d_dh = take(d.dh);
@@ -137,8 +144,16 @@ constexpr int kMxtMinAvg = 48;
 cudaError_t launch_mxt_gemm(const ForwardArgs& a, int w2, const void* tiles, const int* ntiles, int shared_tiles,
                             const MxBuffers& m, cudaStream_t st);
 
+// Shared expert for at least kShMinTokens tokens: int8 weights widened to f16
+// into sh16, then w13 with SwiGLU into hs; w2 with the combine of y_slot fused
+// into its epilogue, writing out.
+bool sh_supported(const v4moe_config& c, int64_t T);
+cudaError_t launch_sh_w13(const ForwardArgs& a, const __half* x16, const int* sigma, char* sh16, cudaStream_t st);
+cudaError_t launch_sh_w2_combine(const ForwardArgs& a, char* sh16, cudaStream_t st);
+
 // Tensor-core path (tcgen05 grouped GEMMs) for larger token counts.
-cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, cudaStream_t st);
+cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, char* sh16,
+                              cudaStream_t st);
 
 // Decode path: the whole layer (routing included in layer mode) as three
 // kernels chained by programmatic dependent launch, for at most

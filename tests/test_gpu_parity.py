@@ -102,6 +102,18 @@ def test_ragged_token_counts_multi_tile(T):
     run_parity(li, _layer(li))
 
 
+@pytest.mark.parametrize("T,routing", [(600, "learned"), (1100, "hash")])
+def test_prefill_sized_ragged(T, routing):
+    """Token-major block-scaled tiles with the shared expert on its own f16
+    GEMM (the combine in its epilogue); ragged last token tiles."""
+    if routing == "hash":
+        wl = IN.Workload("pre_hash", T=T, H=512, E=16, I=512, Is=256, routing="hash", vocab=3000, seed=9)
+    else:
+        wl = IN.Workload("pre_mid", T=T, H=1024, E=32, I=512, Is=512, bias_std=0.05, seed=13)
+    li = IN.make_layer_inputs(wl)
+    run_parity(li, _layer(li))
+
+
 @pytest.mark.parametrize("T", [5, 200])
 def test_hash_routing_small(T):
     wl = IN.Workload("hash_small", T=T, H=512, E=16, I=256, Is=256, routing="hash", vocab=1000,
