@@ -65,6 +65,7 @@ constexpr int kStages13 = 5;
 constexpr int kMaxStages2 = 6;
 constexpr int kNJ = 4;             // K blocks per warp held in registers (K <= 4096)
 constexpr int kMaxHit = 64;        // distinct routed experts of a batch (T * k <= 64)
+constexpr int kShRows = 64;        // shared-expert rows per CTA with preloaded scales
 constexpr uint32_t kBarTries = 1u << 20;
 
 // Control block words (workspace): the routing tables, rewritten by every
@@ -366,25 +367,16 @@ __device__ __noinline__ void write_permutation(RouteSmem& S, const DecParams& P,
 }
 
 // Top-k selection of token t (one warp) from scores and bias in shared memory,
-// into the RouteSmem selection arrays. Out of line: the w13 kernel calls it
-// with its activation fragments live.
-template <int NPER>
-__device__ __noinline__ void select_learned_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
-                                                  const float* sbias) {
-  select_learned_n<false, NPER>(t, P.E, P.k, P.routed_scale, ssc + size_t(t) * P.E, sbias, S.sel_ids, S.sel_w);
-}
-__device__ __noinline__ void select_hash_token(RouteSmem& S, const DecParams& P, int t, const float* ssc) {
-  select_hash_warp<true>(t, P.E, P.k, P.vocab, P.routed_scale, ssc + size_t(t) * P.E, P.token_ids, P.tid2eid,
-                         S.sel_ids, S.sel_w, P.status);
-}
-__device__ __forceinline__ void select_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
+// into the RouteSmem selection arrays.
+__device__ __noinline__ void select_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
                                              const float* sbias) {
   if (P.token_ids)
-    select_hash_token(S, P, t, ssc);
+    select_hash_warp<true>(t, P.E, P.k, P.vocab, P.routed_scale, ssc + size_t(t) * P.E, P.token_ids, P.tid2eid,
+                           S.sel_ids, S.sel_w, P.status);
   else if (P.E <= 256)
-    select_learned_token<8>(S, P, t, ssc, sbias);
+    select_learned_n<false, 8>(t, P.E, P.k, P.routed_scale, ssc + size_t(t) * P.E, sbias, S.sel_ids, S.sel_w);
   else
-    select_learned_token<32>(S, P, t, ssc, sbias);
+    select_learned_n<false, 32>(t, P.E, P.k, P.routed_scale, ssc + size_t(t) * P.E, sbias, S.sel_ids, S.sel_w);
 }
 
 constexpr int kRouteWarps = 8;
@@ -439,6 +431,7 @@ struct W13Smem {
   int lastfill[kStages13];
   int sigma[8];
   uint32_t xmax[2][kGW][8];
+  float sh_scale[2][kShRows];  // gate / up row scales of this CTA's shared slabs
   Tables tb;
   RouteSmem rt;
 };
@@ -513,30 +506,6 @@ __device__ __forceinline__ Chunk w13_chunk(const DecParams& P, int nh, int b, in
   return c;
 }
 
-// Asks L2 for the chunk's shared (routed == false) or routed slabs, as one
-// range per weight tensor and expert (one lane).
-__device__ __forceinline__ void prefetch13(const DecParams& P, const Tables& tb, const Chunk& c, bool routed) {
-  const int H = P.H;
-  if (!routed) {
-    if (c.s1 <= c.s0) return;
-    const char* sh = reinterpret_cast<const char*>(P.sh13);
-    prefetch_l2_range(sh + size_t(4 * c.s0) * H, size_t(4 * (c.s1 - c.s0)) * H);
-    prefetch_l2_range(sh + size_t(P.Is + 4 * c.s0) * H, size_t(4 * (c.s1 - c.s0)) * H);
-    return;
-  }
-  const int i8 = P.I / 8;
-  for (int r = c.r0; r < c.r1;) {
-    const int li = r / i8, re = min(c.r1, (li + 1) * i8);
-    const size_t rows = size_t(8) * (re - r);
-    const size_t rg = size_t(tb.hit[li]) * 2 * P.I + size_t(8) * (r - li * i8), ru = rg + P.I;
-    prefetch_l2_range(P.w13_codes + rg * (H / 2), rows * (H / 2));
-    prefetch_l2_range(P.w13_codes + ru * (H / 2), rows * (H / 2));
-    prefetch_l2_range(P.w13_scales + rg * (H / 32), rows * (H / 32));
-    prefetch_l2_range(P.w13_scales + ru * (H / 32), rows * (H / 32));
-    r = re;
-  }
-}
-
 // The w2 rows of the 16-row output blocks that CTA b of the w2 kernel owns
 // (blocks [b w2_per, (b + 1) w2_per)): the shared expert's, or every routed
 // expert's (one lane).
@@ -578,10 +547,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
   __syncthreads();
   // The w2 kernel may launch now (its CTAs start as these leave their SMs).
   pdl_launch_dependents();
-  // Ask L2 for everything that does not depend on the routing.
-  if (warp == 15 && lane == 0) {
-    prefetch13(P, S.tb, w13_chunk(P, 0, b, G), false);
-    prefetch_w2_share(P, S.tb, b, false);
+  // Global memory outside the ring is read before the first copy or L2
+  // request is issued: on this GPU a global load waits behind the SM's
+  // transfers in flight. The shared slabs' row scales:
+  {
+    const Chunk c0 = w13_chunk(P, 0, b, G);  // the shared range does not depend on the routing
+    for (int i = threadIdx.x; i < 4 * (c0.s1 - c0.s0) && i < kShRows; i += blockDim.x) {
+      S.sh_scale[0][i] = __ldg(P.sh13_scale + 4 * c0.s0 + i);
+      S.sh_scale[1][i] = __ldg(P.sh13_scale + P.Is + 4 * c0.s0 + i);
+    }
   }
 
   const int q = warp / kGW, wi = warp % kGW;
@@ -634,6 +608,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
   float* ssc = reinterpret_cast<float*>(stages);
   float* sbias = ssc + size_t(T) * P.E;
   if (P.layer_mode && !P.token_ids) {
+    // the bias is an input: staged before the wait
+    for (int i = threadIdx.x; i < P.E; i += blockDim.x) sbias[i] = __ldg(P.bias + i);
+    __syncthreads();
     // Run the selection once on whatever the ring holds, results discarded:
     // its code is then cached when the scores arrive.
     if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
@@ -644,8 +621,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
   pdl_wait();
   if (P.layer_mode) {
     for (int i = threadIdx.x; i < T * P.E; i += blockDim.x) ssc[i] = __ldcg(P.scores + i);
-    if (!P.token_ids)
-      for (int i = threadIdx.x; i < P.E; i += blockDim.x) sbias[i] = __ldg(P.bias + i);
     __syncthreads();
     if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
     __syncthreads();
@@ -731,7 +706,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
         }
       }
     } else if (g < 4) {
-      const float sg = __ldg(P.sh13_scale + m.row0 + g), su = __ldg(P.sh13_scale + P.Is + m.row0 + g);
+      const int rl = m.row0 + g - 4 * ch.s0;  // row within this CTA's shared slabs
+      const float sg = rl < kShRows ? S.sh_scale[0][rl] : __ldg(P.sh13_scale + m.row0 + g);
+      const float su = rl < kShRows ? S.sh_scale[1][rl] : __ldg(P.sh13_scale + P.Is + m.row0 + g);
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
         const int tok = 2 * t + qq;
@@ -757,6 +734,7 @@ struct W2Smem {
   uint64_t full[kMaxStages2];
   int redcnt[kMaxStages2];
   int lastfill[kMaxStages2];
+  float sh_scale[kShRows];  // shared-expert row scales of this CTA's output rows
   Tables tb;
 };
 constexpr size_t kHead2 = (sizeof(W2Smem) + 127) / 128 * 128;
@@ -822,6 +800,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
   const int nrb_mine = max(0, min(P.w2_per, P.H / 16 - b * P.w2_per));
   const bool has_sh = P.Is > 0;
 
+  // row scales first: a global load waits behind the SM's copies in flight
+  if (has_sh)
+    for (int i = threadIdx.x; i < 16 * nrb_mine && i < kShRows; i += blockDim.x)
+      S.sh_scale[i] = __ldg(P.sh2_scale + 16 * b * P.w2_per + i);
+  __syncthreads();
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&S.full[s], 1);
@@ -901,7 +884,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
       float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
       if (sh) {
         tile_s8<2, 8>(st + g * P.Is, st + (g + 8) * P.Is, true, 0, nkb, wi, Bf, a0, a1);
-        const float sa = __ldg(P.sh2_scale + m.rb * 16 + g), sb = __ldg(P.sh2_scale + m.rb * 16 + g + 8);
+        const int rl = (m.rb - b * P.w2_per) * 16 + g;  // row within this CTA's output rows
+        const float sa = rl < kShRows ? S.sh_scale[rl] : __ldg(P.sh2_scale + m.rb * 16 + g);
+        const float sb = rl + 8 < kShRows ? S.sh_scale[rl + 8] : __ldg(P.sh2_scale + m.rb * 16 + g + 8);
         acc.x += (a0[0] + a1[0]) * sa;
         acc.y += (a0[1] + a1[1]) * sa;
         acc.z += (a0[2] + a1[2]) * sb;

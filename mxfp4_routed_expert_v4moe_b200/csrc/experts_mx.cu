@@ -48,25 +48,30 @@ namespace {
 constexpr int MBM = 128;       // weight rows per tile
 constexpr int MBK = 128;       // K per stage (4 MMA steps of 32)
 constexpr int MBN = 128;       // max tokens per tile
-constexpr int kMStages = 4;
+constexpr int kMMaxStages = 12;
 constexpr int kMThreads = 384;
 constexpr uint32_t kMTries = 1u << 21;
 
 enum { kMW13 = 0, kMW2 = 1 };
 
-constexpr int kMA = MBM * MBK;   // 16 KB: E2M1 codes expanded to one byte each
-constexpr int kMB = MBN * MBK;   // 16 KB per activation plane
-constexpr int kMOffA = 0;
-constexpr int kMOffBh = kMOffA + kMStages * kMA;
-constexpr int kMOffBl = kMOffBh + kMStages * kMB;
-constexpr int kMOffX = kMOffBl + kMStages * kMB;   // epilogue exchange [128][33] fp32
+// Shared memory: nst stages of [A: 128 weight rows x 128 K, E2M1 codes
+// expanded to one byte each (16 KB)][activation hi plane: bn rows x 128 B]
+// [lo plane], then the epilogue exchange and the barriers. bn (the token
+// tile, a multiple of 32 up to MBN) and nst are chosen per launch: small
+// token tiles leave room for a deeper ring.
+constexpr int kMA = MBM * MBK;
 constexpr int kMXch = 33;
-constexpr int kMOffBar = kMOffX + 128 * kMXch * 4;
-constexpr int kMSmem = kMOffBar + 256 + 1024;
+constexpr int kMXchBytes = 128 * kMXch * 4;  // epilogue exchange [128][33] fp32
+constexpr int kMSmemMax = 232448;           // dynamic shared memory per block
+__host__ __device__ constexpr int mx_stage_bytes(int bn) { return kMA + 2 * bn * MBK; }
+// Scale slot (two of them, each covering four K chunks): 16 bytes per weight
+// row, then per token of the hi and the lo plane, brought in by TMA.
+__host__ __device__ constexpr int mx_scale_slot(int bn) { return 16 * (MBM + 2 * bn); }
 
 // TMEM columns: two accumulators of MBN, then 12 scale columns per stage.
 constexpr uint32_t kMColSF = 2 * MBN;
 constexpr uint32_t kMTmemCols = 512;
+static_assert(kMColSF + 12 * kMMaxStages <= kMTmemCols, "TMEM columns");
 
 struct MxTile {
   int grp, row0, n0, n;
@@ -76,6 +81,8 @@ struct MxParams {
   int T, H, I, E, k;
   float limit;
   int mode;
+  int bn;   // token tile (rows of an activation plane per stage)
+  int nst;  // ring stages
   const int32_t* offsets;
   const MxTile* tiles;
   const int* ntiles;      // tile count of the list (routed tiles come first)
@@ -92,15 +99,52 @@ struct MxParams {
 };
 
 struct MxBars {
-  uint64_t full[kMStages];
-  uint64_t sf_full[kMStages];
-  uint64_t empty[kMStages];
+  uint64_t full[kMMaxStages];
+  uint64_t sf_full[kMMaxStages];
+  uint64_t empty[kMMaxStages];
+  uint64_t sc_full[2];
+  uint64_t sc_empty[2];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t done;
   uint32_t tmem_base;
   int abort;
 };
+
+constexpr int kMBarBytes = (int(sizeof(MxBars)) + 127) / 128 * 128;
+
+// This CTA's tiles (list positions blockIdx.x + i * gridDim.x) with their first
+// activation row, copied into shared memory before the first TMA copy: every
+// role walks them, and on this GPU a global load waits behind the SM's copies
+// in flight. Past kTileCache tiles the list is read from global memory.
+constexpr int kTileCache = 256;
+struct TileCache {
+  MxTile t[kTileCache];
+  int brow0[kTileCache];
+};
+constexpr int kTileCacheBytes = int(sizeof(TileCache));
+
+// Whole CTA; returns the number of this CTA's tiles.
+__device__ __forceinline__ int cache_tiles(const MxParams& P, int ntiles, TileCache& C) {
+  const int nmine = int(blockIdx.x) < ntiles ? (ntiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
+  for (int i = threadIdx.x; i < nmine && i < kTileCache; i += blockDim.x) {
+    const MxTile t = P.tiles[blockIdx.x + i * gridDim.x];
+    C.t[i] = t;
+    C.brow0[i] = P.offsets[t.grp] + t.n0;
+  }
+  __syncthreads();
+  return nmine;
+}
+
+__device__ __forceinline__ MxTile tile_at(const MxParams& P, const TileCache& C, int i, int& brow0) {
+  if (i < kTileCache) {
+    brow0 = C.brow0[i];
+    return C.t[i];
+  }
+  const MxTile t = P.tiles[blockIdx.x + i * gridDim.x];
+  brow0 = P.offsets[t.grp] + t.n0;
+  return t;
+}
 
 __device__ __forceinline__ bool mwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status) {
   for (uint32_t i = 0; i < kMTries; ++i) {
@@ -227,7 +271,7 @@ struct MxGeo {
   int wrow0, wrow1;    // first weight rows of the two 64-row halves
 };
 
-__device__ __forceinline__ MxGeo mx_geo(const MxParams& P, const MxTile& t) {
+__device__ __forceinline__ MxGeo mx_geo(const MxParams& P, const MxTile& t, int brow0) {
   MxGeo g;
   g.n = t.n;
   g.n_load = (t.n + 31) / 32 * 32;
@@ -243,11 +287,9 @@ __device__ __forceinline__ MxGeo mx_geo(const MxParams& P, const MxTile& t) {
     g.wrow1 = g.wrow0 + 64;
   }
   g.nk = g.K / MBK;
-  g.brow0 = P.offsets[t.grp] + t.n0;
+  g.brow0 = brow0;
   return g;
 }
-
-__device__ __forceinline__ int t_grp(const MxParams& P, int ti) { return P.tiles[ti].grp; }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
   asm volatile(
@@ -284,10 +326,15 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 __global__ void __launch_bounds__(kMThreads, 1)
     k_mx_gemm(MxParams P, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmBh,
-              const __grid_constant__ CUtensorMap tmBl) {
+              const __grid_constant__ CUtensorMap tmBl, const __grid_constant__ CUtensorMap tmSw,
+              const __grid_constant__ CUtensorMap tmSh, const __grid_constant__ CUtensorMap tmSl) {
   extern __shared__ __align__(1024) char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  MxBars& B = *reinterpret_cast<MxBars*>(smem + kMOffBar);
+  const int kMStages = P.nst, stage = mx_stage_bytes(P.bn);
+  const int kMOffSc = kMStages * stage, slot = mx_scale_slot(P.bn);
+  const int kMOffX = kMOffSc + 2 * slot;
+  MxBars& B = *reinterpret_cast<MxBars*>(smem + kMOffX + kMXchBytes);
+  TileCache& TC = *reinterpret_cast<TileCache*>(smem + kMOffX + kMXchBytes + kMBarBytes);
   volatile int* abort_flag = &B.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -300,6 +347,8 @@ __global__ void __launch_bounds__(kMThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&B.acc_full[b], 1);
       mbar_init(&B.acc_empty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&B.sc_full[b], 1);
+      mbar_init(&B.sc_empty[b], 4);   // one arrival per scale-writer warp
     }
     mbar_init(&B.done, 1);
     B.abort = 0;
@@ -314,18 +363,41 @@ __global__ void __launch_bounds__(kMThreads, 1)
   tc_fence_after();
   const uint32_t tmem = B.tmem_base;
   pdl_wait();  // tiles, routing and activations come from earlier kernels
-  const int ntiles = *P.ntiles - P.shared_tiles;
+  const int nmine = cache_tiles(P, *P.ntiles - P.shared_tiles, TC);
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmBh);
     prefetch_tmap(&tmBl);
-    uint32_t gc = 0;
+    prefetch_tmap(&tmSw);
+    prefetch_tmap(&tmSh);
+    prefetch_tmap(&tmSl);
+    uint32_t gc = 0, gs = 0;
     bool ok = true;
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
-      const MxGeo g = mx_geo(P, P.tiles[ti]);
+    for (int li = 0; li < nmine && ok; ++li) {
+      int brow0;
+      const MxTile t = tile_at(P, TC, li, brow0);
+      const MxGeo g = mx_geo(P, t, brow0);
       for (int c = 0; c < g.nk; ++c, ++gc) {
+        if ((c & 3) == 0) {  // scales of this chunk and the next three
+          const uint32_t j = gs & 1u, v = gs >> 1;
+          if (!mwait(&B.sc_empty[j], (v & 1u) ^ 1u, abort_flag, P.status)) {
+            ok = false;
+            break;
+          }
+          char* sc = smem + kMOffSc + j * slot;
+          mbar_arrive_expect_tx(&B.sc_full[j], uint32_t(16 * (MBM + 2 * g.n_load)));
+          if (P.mode == kMW13)
+            tma_load_3d(sc, &tmSw, c * 4, g.wrow0 - g.ebase, 2 * t.grp, &B.sc_full[j]);
+          else
+            tma_load_2d(sc, &tmSw, c * 4, g.wrow0, &B.sc_full[j]);
+          for (int i = 0; i < g.n_load / 32; ++i) {
+            tma_load_2d(sc + 16 * MBM + 512 * i, &tmSh, c * 4, g.brow0 + 32 * i, &B.sc_full[j]);
+            tma_load_2d(sc + 16 * (MBM + P.bn) + 512 * i, &tmSl, c * 4, g.brow0 + 32 * i, &B.sc_full[j]);
+          }
+          ++gs;
+        }
         const int s = gc % kMStages;
         const uint32_t u = gc / kMStages;
         if (!mwait(&B.empty[s], (u & 1u) ^ 1u, abort_flag, P.status)) {
@@ -333,28 +405,35 @@ __global__ void __launch_bounds__(kMThreads, 1)
           break;
         }
         // E2M1 rows count their packed bytes (64 per row and chunk); the
-        // activation boxes are always 128 rows (rows past the tile's tokens
-        // only feed columns the epilogue ignores).
-        mbar_arrive_expect_tx(&B.full[s], uint32_t(MBM * MBK / 2 + 2 * MBN * MBK));
-        char* as = smem + kMOffA + s * kMA;
+        // activation planes come in boxes of 32 rows, as many as the tile's
+        // tokens need (rows past them only feed columns the epilogue ignores).
+        mbar_arrive_expect_tx(&B.full[s], uint32_t(MBM * MBK / 2 + 2 * g.n_load * MBK));
+        char* as = smem + s * stage;
         if (P.mode == kMW13)  // gate and up halves in one box of the 3-D map
-          tma_load_3d(as, &tmA, c * MBK, g.wrow0 - g.ebase, 2 * t_grp(P, ti), &B.full[s]);
+          tma_load_3d(as, &tmA, c * MBK, g.wrow0 - g.ebase, 2 * t.grp, &B.full[s]);
         else
           tma_load_2d(as, &tmA, c * MBK, g.wrow0, &B.full[s]);
-        tma_load_2d(smem + kMOffBh + s * kMB, &tmBh, c * MBK, g.brow0, &B.full[s]);
-        tma_load_2d(smem + kMOffBl + s * kMB, &tmBl, c * MBK, g.brow0, &B.full[s]);
+        for (int i = 0; i < g.n_load / 32; ++i) {
+          tma_load_2d(as + kMA + i * 32 * MBK, &tmBh, c * MBK, g.brow0 + 32 * i, &B.full[s]);
+          tma_load_2d(as + kMA + P.bn * MBK + i * 32 * MBK, &tmBl, c * MBK, g.brow0 + 32 * i, &B.full[s]);
+        }
       }
     }
     for (uint32_t q = 0; q < uint32_t(kMStages) && q < gc; ++q) {
       const uint32_t gq = gc - 1 - q;
       mbar_wait_bounded(&B.full[gq % kMStages], (gq / kMStages) & 1u, kMTries);
     }
+    for (uint32_t q = 0; q < 2u && q < gs; ++q) {
+      const uint32_t gq = gs - 1 - q;
+      mbar_wait_bounded(&B.sc_full[gq & 1u], (gq >> 1) & 1u, kMTries);
+    }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     uint32_t gc = 0, lt = 0;
     bool ok = true;
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x, ++lt) {
-      const MxGeo g = mx_geo(P, P.tiles[ti]);
+    for (int li = 0; li < nmine && ok; ++li, ++lt) {
+      int brow0;
+      const MxGeo g = mx_geo(P, tile_at(P, TC, li, brow0), brow0);
       const uint32_t b = lt & 1u, v = lt >> 1;
       if (!mwait(&B.acc_empty[b], (v & 1u) ^ 1u, abort_flag, P.status)) break;
       tc_fence_after();
@@ -369,9 +448,9 @@ __global__ void __launch_bounds__(kMThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(smem + kMOffA + s * kMA);
-        const uint32_t bh0 = smem_u32(smem + kMOffBh + s * kMB);
-        const uint32_t bl0 = smem_u32(smem + kMOffBl + s * kMB);
+        const uint32_t a0 = smem_u32(smem + s * stage);
+        const uint32_t bh0 = a0 + kMA;
+        const uint32_t bl0 = bh0 + P.bn * MBK;
         const uint32_t sf = tmem + kMColSF + 12u * uint32_t(s);
 #pragma unroll
         for (int kk = 0; kk < MBK / 32; ++kk) {
@@ -391,70 +470,51 @@ __global__ void __launch_bounds__(kMThreads, 1)
     mbar_wait_bounded(&B.done, 0, kMTries);
   } else if (warp >= 8) {
     // ------------------------------------------------------------ scale writers
-    // One 16-byte load per row (weights) or token (both planes) covers four
-    // chunks; the next four chunks' loads are in flight while these are used.
+    // The scales of four chunks arrive by TMA in a scale slot (a global load
+    // here would wait behind the SM's copies in flight); per chunk each warp
+    // moves its lane quarter's copy into TMEM.
     const int q = warp - 8;  // TMEM lane quarter of this warp (warp % 4)
-    uint32_t gc = 0;
+    uint32_t gc = 0, gs = 0;
     bool ok = true;
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
-      const MxTile t = P.tiles[ti];
-      const MxGeo g = mx_geo(P, t);
-      const int G16 = g.K / 512;  // 16-byte scale words per row
-      const uint4* wr[4];
-      const uint4* th[4];
-      const uint4* tl[4];
-      bool tv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = lane + 32 * i;
-        wr[i] = reinterpret_cast<const uint4*>(P.w_scales) + size_t(r < 64 ? g.wrow0 + r : g.wrow1 + (r - 64)) * G16;
-        const int n = min(r, g.n - 1);
-        th[i] = reinterpret_cast<const uint4*>(P.b_sc_hi) + size_t(g.brow0 + n) * G16;
-        tl[i] = reinterpret_cast<const uint4*>(P.b_sc_lo) + size_t(g.brow0 + n) * G16;
-        tv[i] = r < g.n_mma;
-      }
-      uint4 ca[4], ch[4], cl[4], na[4], nh[4], nl[4];
-      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        ca[i] = __ldg(wr[i]);
-        ch[i] = tv[i] ? __ldg(th[i]) : z;
-        cl[i] = tv[i] ? __ldg(tl[i]) : z;
-      }
-      for (int g4 = 0; g4 < G16 && ok; ++g4) {
-        if (g4 + 1 < G16) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            na[i] = __ldg(wr[i] + g4 + 1);
-            nh[i] = tv[i] ? __ldg(th[i] + g4 + 1) : z;
-            nl[i] = tv[i] ? __ldg(tl[i] + g4 + 1) : z;
-          }
+    for (int li = 0; li < nmine && ok; ++li) {
+      int brow0;
+      const MxTile t = tile_at(P, TC, li, brow0);
+      const MxGeo g = mx_geo(P, t, brow0);
+      for (int c = 0; c < g.nk && ok; ++c, ++gc) {
+        const uint32_t j = gs & 1u;
+        if ((c & 3) == 0 && !__all_sync(0xffffffffu, mwait(&B.sc_full[j], (gs >> 1) & 1u, abort_flag, P.status))) {
+          ok = false;
+          break;
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j, ++gc) {
-          const int s = gc % kMStages;
-          const uint32_t u = gc / kMStages;
-          if (!mwait(&B.empty[s], (u & 1u) ^ 1u, abort_flag, P.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          auto wj = [j](const uint4& v) { return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w; };
-          const uint32_t sf = tmem + kMColSF + 12u * uint32_t(s) + (uint32_t(32 * q) << 16);
-          tmem_st_32x32b_x4(sf, wj(ca[0]), wj(ca[1]), wj(ca[2]), wj(ca[3]));
-          tmem_st_32x32b_x4(sf + 4, wj(ch[0]), wj(ch[1]), wj(ch[2]), wj(ch[3]));
-          tmem_st_32x32b_x4(sf + 8, wj(cl[0]), wj(cl[1]), wj(cl[2]), wj(cl[3]));
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&B.sf_full[s]);
+        const int s = gc % kMStages;
+        const uint32_t u = gc / kMStages;
+        if (!__all_sync(0xffffffffu, mwait(&B.empty[s], (u & 1u) ^ 1u, abort_flag, P.status))) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        // row 32 i + lane of each operand, the four bytes of this chunk
+        const char* sc = smem + kMOffSc + j * slot + 4 * (c & 3);
+        uint32_t wa[4], hv[4], lv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          ca[i] = na[i];
-          ch[i] = nh[i];
-          cl[i] = nl[i];
+          const int r = 32 * i + lane;
+          wa[i] = *reinterpret_cast<const uint32_t*>(sc + 16 * r);
+          hv[i] = r < g.n_mma ? *reinterpret_cast<const uint32_t*>(sc + 16 * (MBM + r)) : 0u;
+          lv[i] = r < g.n_mma ? *reinterpret_cast<const uint32_t*>(sc + 16 * (MBM + P.bn + r)) : 0u;
         }
+        const uint32_t sf = tmem + kMColSF + 12u * uint32_t(s) + (uint32_t(32 * q) << 16);
+        tmem_st_32x32b_x4(sf, wa[0], wa[1], wa[2], wa[3]);
+        tmem_st_32x32b_x4(sf + 4, hv[0], hv[1], hv[2], hv[3]);
+        tmem_st_32x32b_x4(sf + 8, lv[0], lv[1], lv[2], lv[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&B.sf_full[s]);
+          if ((c & 3) == 3) mbar_arrive(&B.sc_empty[j]);
+        }
+        if ((c & 3) == 3) ++gs;
       }
     }
   } else if (warp >= 4) {
@@ -462,9 +522,10 @@ __global__ void __launch_bounds__(kMThreads, 1)
     const int q = warp - 4;  // TMEM lane quarter
     float* xch = reinterpret_cast<float*>(smem + kMOffX);
     uint32_t lt = 0;
-    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x, ++lt) {
-      const MxTile t = P.tiles[ti];
-      const MxGeo g = mx_geo(P, t);
+    for (int li = 0; li < nmine; ++li, ++lt) {
+      int brow0;
+      const MxTile t = tile_at(P, TC, li, brow0);
+      const MxGeo g = mx_geo(P, t, brow0);
       const uint32_t b = lt & 1u, v = lt >> 1;
       const int row = 32 * q + lane;
       const bool got = mwait(&B.acc_full[b], v & 1u, abort_flag, P.status);
@@ -562,7 +623,9 @@ constexpr int kXScL = kXScH + XM * 16;
 constexpr int kXSc = kXScL + XM * 16;   // 8 KB
 constexpr int kXOffSc = kXStages * kXStage;
 constexpr int kXOffBar = kXOffSc + 2 * kXSc;
-constexpr int kXSmem = kXOffBar + 256 + 1024;
+constexpr int kXOffTiles = kXOffBar + 256;
+constexpr int kXSmem = kXOffTiles + kTileCacheBytes + 1024;
+static_assert(kXSmem <= kMSmemMax, "dynamic shared memory per block");
 constexpr uint32_t kXColSF = XN;        // per stage 16 columns: SFA hi (4), SFA lo (4), SFB (8)
 constexpr uint32_t kXTmemCols = 512;
 
@@ -584,10 +647,10 @@ struct XGeo {
   int wy, wz;    // weight coordinates: w13 (channel, 2 expert), w2 (row, unused)
 };
 
-__device__ __forceinline__ XGeo xgeo(const MxParams& P, const MxTile& t) {
+__device__ __forceinline__ XGeo xgeo(const MxParams& P, const MxTile& t, int brow0) {
   XGeo g;
   g.n = t.n;
-  g.brow0 = P.offsets[t.grp] + t.n0;
+  g.brow0 = brow0;
   if (P.mode == kMW13) {
     g.K = P.H;
     g.wy = t.row0;
@@ -619,6 +682,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
   extern __shared__ __align__(1024) char smem_raw[];
   char* smem = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   XBars& B = *reinterpret_cast<XBars*>(smem + kXOffBar);
+  TileCache& TC = *reinterpret_cast<TileCache*>(smem + kXOffTiles);
   volatile int* abort_flag = &B.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool w13 = P.mode == kMW13;
@@ -648,7 +712,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
   tc_fence_after();
   const uint32_t tmem = B.tmem_base;
   pdl_wait();  // tiles, routing and activations come from earlier kernels
-  const int ntiles = *P.ntiles - P.shared_tiles;
+  const int nmine = cache_tiles(P, *P.ntiles - P.shared_tiles, TC);
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -660,8 +724,9 @@ __global__ void __launch_bounds__(kXThreads, 1)
     prefetch_tmap(&tmSl);
     uint32_t gc = 0, gs = 0;
     bool ok = true;
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
-      const XGeo g = xgeo(P, P.tiles[ti]);
+    for (int li = 0; li < nmine && ok; ++li) {
+      int brow0;
+      const XGeo g = xgeo(P, tile_at(P, TC, li, brow0), brow0);
       for (int c = 0; c < g.nk; ++c, ++gc) {
         if ((c & 3) == 0) {  // scales of this chunk and the next three
           const uint32_t j = gs & 1u, v = gs >> 1;
@@ -710,8 +775,9 @@ __global__ void __launch_bounds__(kXThreads, 1)
     uint32_t gc = 0, lt = 0;
     bool ok = true;
     const uint32_t idesc = idesc_mxt(XM, XN);
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x, ++lt) {
-      const XGeo g = xgeo(P, P.tiles[ti]);
+    for (int li = 0; li < nmine && ok; ++li, ++lt) {
+      int brow0;
+      const XGeo g = xgeo(P, tile_at(P, TC, li, brow0), brow0);
       if (!mwait(&B.acc_empty, (lt & 1u) ^ 1u, abort_flag, P.status)) break;
       tc_fence_after();
       for (int c = 0; c < g.nk; ++c, ++gc) {
@@ -751,8 +817,9 @@ __global__ void __launch_bounds__(kXThreads, 1)
     const int q = warp & 3;
     uint32_t gc = 0, gs = 0;
     bool ok = true;
-    for (int ti = blockIdx.x; ti < ntiles && ok; ti += gridDim.x) {
-      const XGeo g = xgeo(P, P.tiles[ti]);
+    for (int li = 0; li < nmine && ok; ++li) {
+      int brow0;
+      const XGeo g = xgeo(P, tile_at(P, TC, li, brow0), brow0);
       for (int c = 0; c < g.nk && ok; ++c, ++gc) {
         const uint32_t j = gs & 1u;
         if ((c & 3) == 0 && !__all_sync(0xffffffffu, mwait(&B.sc_full[j], (gs >> 1) & 1u, abort_flag, P.status))) {
@@ -795,9 +862,10 @@ __global__ void __launch_bounds__(kXThreads, 1)
     const int sub = (warp - kXFirstEpi) >> 2;  // quarter of the columns
     const int row = 32 * q + lane;
     uint32_t lt = 0;
-    for (int ti = blockIdx.x; ti < ntiles; ti += gridDim.x, ++lt) {
-      const MxTile t = P.tiles[ti];
-      const XGeo g = xgeo(P, t);
+    for (int li = 0; li < nmine; ++li, ++lt) {
+      int brow0;
+      const MxTile t = tile_at(P, TC, li, brow0);
+      const XGeo g = xgeo(P, t, brow0);
       if (!__all_sync(0xffffffffu, mwait(&B.acc_full, lt & 1u, abort_flag, P.status)) || *abort_flag) break;
       tc_fence_after();
       const uint32_t acc = tmem + (uint32_t(32 * q) << 16);
@@ -961,7 +1029,7 @@ cudaError_t launch_mx_gather(const ForwardArgs& a, __half* x16, int* sigma, cons
 }
 
 cudaError_t launch_mx_gemm(const ForwardArgs& a, int w2, const void* tiles, const int* ntiles, int shared_tiles,
-                           const MxBuffers& m, cudaStream_t st) {
+                           int bn, const MxBuffers& m, cudaStream_t st) {
   const v4moe_config& c = a.c;
   const int64_t S = int64_t(a.T) * c.top_k;
   MxParams P;
@@ -982,31 +1050,45 @@ cudaError_t launch_mx_gemm(const ForwardArgs& a, int w2, const void* tiles, cons
   P.hs_lo = m.hs_lo;
   P.y_slot = a.y_slot;
   P.status = a.status;
-  CUtensorMap mA, mBh, mBl;
+  CUtensorMap mA, mBh, mBl, mSw, mSh, mSl;
   bool ok = true;
+  constexpr auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  constexpr auto NS = CU_TENSOR_MAP_SWIZZLE_NONE;
+  const uint64_t H = c.hidden, I = c.inter, E = c.n_experts;
   if (!w2) {
     P.w_scales = a.w.w13_scales;
     P.b_sc_hi = m.xs_hi;
     P.b_sc_lo = m.xs_lo;
+    ok &= mx_map3d(&mSw, a.w.w13_scales, U8, H / 32, H / 32, I, 2 * E, 16, MBM / 2, NS);
+    ok &= mx_map2d(&mSh, m.xs_hi, U8, H / 32, H / 32, S, 16, 32, NS);
+    ok &= mx_map2d(&mSl, m.xs_lo, U8, H / 32, H / 32, S, 16, 32, NS);
     ok &= mx_map_w13(&mA, a.w.w13_codes, c.hidden, c.inter, uint64_t(c.n_experts) * 2);
-    ok &= mx_map(&mBh, m.xq_hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.hidden, c.hidden, S, MBN);
-    ok &= mx_map(&mBl, m.xq_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.hidden, c.hidden, S, MBN);
+    ok &= mx_map(&mBh, m.xq_hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.hidden, c.hidden, S, 32);
+    ok &= mx_map(&mBl, m.xq_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.hidden, c.hidden, S, 32);
   } else {
     P.w_scales = a.w.w2_scales;
     P.b_sc_hi = m.hs_hi;
     P.b_sc_lo = m.hs_lo;
+    ok &= mx_map2d(&mSw, a.w.w2_scales, U8, I / 32, I / 32, E * H, 16, MBM, NS);
+    ok &= mx_map2d(&mSh, m.hs_hi, U8, I / 32, I / 32, S, 16, 32, NS);
+    ok &= mx_map2d(&mSl, m.hs_lo, U8, I / 32, I / 32, S, 16, 32, NS);
     ok &= mx_map(&mA, a.w.w2_codes, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, c.inter, c.inter / 2,
                  uint64_t(c.n_experts) * c.hidden, MBM);
-    ok &= mx_map(&mBh, m.hq_hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.inter, c.inter, S, MBN);
-    ok &= mx_map(&mBl, m.hq_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.inter, c.inter, S, MBN);
+    ok &= mx_map(&mBh, m.hq_hi, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.inter, c.inter, S, 32);
+    ok &= mx_map(&mBl, m.hq_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.inter, c.inter, S, 32);
   }
   if (!ok) return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  set_smem(k_mx_gemm, kMSmem);
-  return launch_kernel(w2 ? "mx_w2" : "mx_w13", k_mx_gemm, dim3(sms), dim3(kMThreads), kMSmem, st, true, P, mA, mBh,
-                       mBl);
+  // as many stages as fit next to the epilogue exchange and the barriers
+  P.bn = bn;
+  const int fixed = 2 * mx_scale_slot(bn) + kMXchBytes + kMBarBytes + kTileCacheBytes + 1024;
+  P.nst = std::min(kMMaxStages, (kMSmemMax - fixed) / mx_stage_bytes(bn));
+  const int smem = P.nst * mx_stage_bytes(bn) + fixed;
+  set_smem(k_mx_gemm, smem);
+  return launch_kernel(w2 ? "mx_w2" : "mx_w13", k_mx_gemm, dim3(sms), dim3(kMThreads), smem, st, true, P, mA, mBh,
+                       mBl, mSw, mSh, mSl);
 }
 
 cudaError_t launch_mxt_gemm(const ForwardArgs& a, int w2, const void* tiles, const int* ntiles, int shared_tiles,

@@ -545,7 +545,7 @@ __device__ __forceinline__ int block_excl_scan_1024(int v, int* warp_tot, int* t
   return warp_tot[warp] + incl - v;
 }
 
-__global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, int Is, int rb13, int rb2,
+__global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, int Is, int rb13, int rb2, int tn,
                                                    const int32_t* __restrict__ offsets,
                                                    TcTile* __restrict__ t13, int* __restrict__ n13, TcTile* __restrict__ t2,
                                                    int* __restrict__ n2) {
@@ -558,7 +558,8 @@ __global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, i
     const int g = threadIdx.x + q * 1024;
     if (g < G) {
       const int n = g < E ? offsets[g + 1] - offsets[g] : T;
-      const int tt = (n + BN - 1) / BN;
+      const int tile = g < E ? tn : BN;
+      const int tt = (n + tile - 1) / tile;
       gn[g] = n;
       c13[q] = tt * (g < E ? I / rb13 : Is / 64);
       c2[q] = tt * (g < E ? H / rb2 : H / 128);
@@ -585,16 +586,17 @@ __global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, i
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int g = warp; g < G; g += 32) {
     const int n = gn[g];
-    const int tt = (n + BN - 1) / BN;
+    const int tile = g < E ? tn : BN;
+    const int tt = (n + tile - 1) / tile;
     const int r13 = g < E ? rb13 : 64, r2 = g < E ? rb2 : 128;
     const int nb13 = (g < E ? I : Is) / r13, nb2 = H / r2;
     for (int i = lane; i < tt * nb13; i += 32) {
-      const int n0 = (i / nb13) * BN;
-      t13[gb13[g] + i] = TcTile{g, (i % nb13) * r13, n0, min(BN, n - n0)};
+      const int n0 = (i / nb13) * tile;
+      t13[gb13[g] + i] = TcTile{g, (i % nb13) * r13, n0, min(tile, n - n0)};
     }
     for (int i = lane; i < tt * nb2; i += 32) {
-      const int n0 = (i / nb2) * BN;
-      t2[gb2[g] + i] = TcTile{g, (i % nb2) * r2, n0, min(BN, n - n0)};
+      const int n0 = (i / nb2) * tile;
+      t2[gb2[g] + i] = TcTile{g, (i % nb2) * r2, n0, min(tile, n - n0)};
     }
   }
 }
@@ -630,11 +632,17 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
 
 }  // namespace
 
+// Token tiles of the lists: at most S / kMxSmallTile + E routed ones (each
+// expert's partial tile) plus the shared expert's T / BN (+ 1).
+static int64_t tile_rows(const v4moe_config& c, int64_t T) {
+  const int64_t S = T * c.top_k;
+  return (S + kMxSmallTile - 1) / kMxSmallTile + c.n_experts + (T + BN - 1) / BN + 2;
+}
+
 size_t tc_extra_bytes(const v4moe_config& c, int64_t T) {
   const int64_t S = T * c.top_k;
-  const int64_t tiles13 = ((S + BN - 1) / BN + c.n_experts + (T + BN - 1) / BN + 2) *
-                          (std::max(c.inter, c.shared_inter) / 64);
-  const int64_t tiles2 = ((S + BN - 1) / BN + c.n_experts + (T + BN - 1) / BN + 2) * (c.hidden / 128);
+  const int64_t tiles13 = tile_rows(c, T) * (std::max(c.inter, c.shared_inter) / 64);
+  const int64_t tiles2 = tile_rows(c, T) * (c.hidden / 128);
   return align_up(size_t(S) * c.hidden * 2) + align_up(size_t(tiles13) * sizeof(TcTile)) +
          align_up(size_t(tiles2) * sizeof(TcTile)) + 256 + 2 * align_up(size_t(S) * (c.hidden / 32)) +
          2 * align_up(size_t(S) * (c.inter / 32));
@@ -647,11 +655,10 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   const int64_t S = int64_t(T) * c.top_k;
   __half* xperm = reinterpret_cast<__half*>(extra);
   char* p = extra + align_up(size_t(S) * c.hidden * 2);
-  const int64_t tiles13 = ((S + BN - 1) / BN + c.n_experts + (T + BN - 1) / BN + 2) *
-                          (std::max(c.inter, c.shared_inter) / 64);
+  const int64_t tiles13 = tile_rows(c, T) * (std::max(c.inter, c.shared_inter) / 64);
   TcTile* t13 = reinterpret_cast<TcTile*>(p);
   p += align_up(size_t(tiles13) * sizeof(TcTile));
-  const int64_t tiles2 = ((S + BN - 1) / BN + c.n_experts + (T + BN - 1) / BN + 2) * (c.hidden / 128);
+  const int64_t tiles2 = tile_rows(c, T) * (c.hidden / 128);
   TcTile* t2 = reinterpret_cast<TcTile*>(p);
   p += align_up(size_t(tiles2) * sizeof(TcTile));
   int* counts = reinterpret_cast<int*>(p);  // [0] = n13, [1] = n2
@@ -685,8 +692,10 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   // Token-major block-scaled tiles (128 slots x 256 weight rows) once the
   // experts average enough tokens to fill them; weight-major ones otherwise.
   const bool mxt = mx && int64_t(T) * c.top_k >= int64_t(kMxtMinAvg) * c.n_experts;
+  // token tile of the routed groups: small for weight-major tiles of few tokens
+  const int tn = mx && !mxt && int64_t(T) * c.top_k < int64_t(kMxSmallAvg) * c.n_experts ? kMxSmallTile : BN;
   e = launch_kernel("tc_tiles", k_tc_tiles, dim3(1), dim3(1024), 0, st, false, T, c.n_experts, c.hidden, c.inter,
-                    shx ? 0 : c.shared_inter, mxt ? 128 : 64, mxt ? 256 : 128, a.offsets, t13, counts, t2,
+                    shx ? 0 : c.shared_inter, mxt ? 128 : 64, mxt ? 256 : 128, tn, a.offsets, t13, counts, t2,
                     counts + 1);
   if (e != cudaSuccess) return e;
 
@@ -750,7 +759,8 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   P.w_scales = a.w.w13_scales;
   P.sh_scale = a.w.sh_w13_scale;
   if (mx) {
-    e = mxt ? launch_mxt_gemm(a, 0, t13, counts, sh13, mb, st) : launch_mx_gemm(a, 0, t13, counts, sh13, mb, st);
+    e = mxt ? launch_mxt_gemm(a, 0, t13, counts, sh13, mb, st)
+            : launch_mx_gemm(a, 0, t13, counts, sh13, tn, mb, st);
     if (e != cudaSuccess) return e;
     P.tail_tiles = sh13;
     if (shx && (e = launch_sh_w13(a, x16, sigma, sh16, st)) != cudaSuccess) return e;
@@ -771,7 +781,8 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   P.w_scales = a.w.w2_scales;
   P.sh_scale = a.w.sh_w2_scale;
   if (mx) {
-    e = mxt ? launch_mxt_gemm(a, 1, t2, counts + 1, sh2, mb, st) : launch_mx_gemm(a, 1, t2, counts + 1, sh2, mb, st);
+    e = mxt ? launch_mxt_gemm(a, 1, t2, counts + 1, sh2, mb, st)
+            : launch_mx_gemm(a, 1, t2, counts + 1, sh2, tn, mb, st);
     if (e != cudaSuccess) return e;
     P.tail_tiles = sh2;
     if (shx) return launch_sh_w2_combine(a, sh16, st);  // the combine is in its epilogue

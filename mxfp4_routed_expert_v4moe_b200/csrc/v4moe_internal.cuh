@@ -135,9 +135,12 @@ struct MxBuffers {
 bool mx_supported(const v4moe_config& c, const v4moe_weights& w);
 cudaError_t launch_mx_gather(const ForwardArgs& a, __half* x16, int* sigma, const MxBuffers& m, cudaStream_t st);
 // tiles: the tensor-core path's tile list (routed tiles first, shared_tiles
-// trailing ones skipped).
+// trailing ones skipped), token tiles of at most bn slots (32, 64 or 128).
+// Few tokens per expert: the small token tile leaves room for a deeper ring.
+constexpr int kMxSmallTile = 32;
+constexpr int kMxSmallAvg = 16;  // slots per expert below which the small tile is used
 cudaError_t launch_mx_gemm(const ForwardArgs& a, int w2, const void* tiles, const int* ntiles, int shared_tiles,
-                           const MxBuffers& m, cudaStream_t st);
+                           int bn, const MxBuffers& m, cudaStream_t st);
 // Token-major variant (128 slots x 256 weight rows per tile), for experts that
 // average at least kMxtMinAvg tokens.
 constexpr int kMxtMinAvg = 48;
