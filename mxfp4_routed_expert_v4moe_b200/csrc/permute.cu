@@ -124,15 +124,39 @@ __global__ void __launch_bounds__(1024) k_perm_scan(int E, int nchunks, const in
   if (threadIdx.x == 0) offsets[E] = total;
 }
 
-__global__ void __launch_bounds__(32) k_perm_scatter(int S, int E, const int32_t* __restrict__ ids,
-                                                     const int32_t* __restrict__ chunk_base,
-                                                     int32_t* __restrict__ sorted_slot,
-                                                     int32_t* __restrict__ slot_pos) {
-  __shared__ int cursor[1024];
-  for (int e = threadIdx.x; e < E; e += 32) cursor[e] = chunk_base[size_t(blockIdx.x) * E + e];
+// One CTA per chunk, its 8 warps on consecutive sub-chunks of kPermChunk / 8
+// slots: per-warp histograms give each warp its starting position per expert
+// (the chunk's base plus the counts of the earlier sub-chunks), so the order
+// stays the stable slot order.
+constexpr int kScatterWarps = 8;
+constexpr int kSubChunk = kPermChunk / kScatterWarps;
+
+__global__ void __launch_bounds__(32 * kScatterWarps) k_perm_scatter(int S, int E, const int32_t* __restrict__ ids,
+                                                                    const int32_t* __restrict__ chunk_base,
+                                                                    int32_t* __restrict__ sorted_slot,
+                                                                    int32_t* __restrict__ slot_pos) {
+  extern __shared__ int pss[];  // [kScatterWarps][E] counts, then cursors
+  const int warp = threadIdx.x >> 5;
+  const int s0 = blockIdx.x * kPermChunk + warp * kSubChunk;
+  const int s1 = min(S, s0 + kSubChunk);
+  int* cnt = pss + warp * E;
+  for (int e = threadIdx.x & 31; e < E; e += 32) cnt[e] = 0;
   __syncwarp();
-  const int s0 = blockIdx.x * kPermChunk, s1 = min(S, s0 + kPermChunk);
-  warp_stable_scatter(ids, s0, s1, E, cursor, sorted_slot, slot_pos);
+  for (int s = s0 + (threadIdx.x & 31); s < s1; s += 32) {
+    const int e = ids[s];
+    if (id_ok(e, E)) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = chunk_base[size_t(blockIdx.x) * E + e];
+    for (int w = 0; w < kScatterWarps; ++w) {
+      const int c = pss[w * E + e];
+      pss[w * E + e] = run;  // becomes warp w's cursor
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (s0 < s1) warp_stable_scatter(ids, s0, s1, E, cnt, sorted_slot, slot_pos);
 }
 
 }  // namespace
@@ -152,8 +176,10 @@ cudaError_t launch_permute(const v4moe_config& c, int T, const int32_t* topk_ids
   e = launch_kernel("perm_scan", k_perm_scan, dim3(1), dim3(1024), 0, st, false, E, nchunks,
                     (const int32_t*)chunk_counts, chunk_base, counts, offsets);
   if (e != cudaSuccess) return e;
-  return launch_kernel("perm_scatter", k_perm_scatter, dim3(nchunks), dim3(32), 0, st, false, S, E, topk_ids,
-                       (const int32_t*)chunk_base, sorted_slot, slot_pos);
+  const size_t smem = size_t(kScatterWarps) * E * sizeof(int);
+  set_smem(k_perm_scatter, smem);
+  return launch_kernel("perm_scatter", k_perm_scatter, dim3(nchunks), dim3(32 * kScatterWarps), smem, st, false, S,
+                       E, topk_ids, (const int32_t*)chunk_base, sorted_slot, slot_pos);
 }
 
 }  // namespace v4moe

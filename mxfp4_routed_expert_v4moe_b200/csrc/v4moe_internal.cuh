@@ -25,6 +25,11 @@ constexpr int kPermChunk = 2048;
 
 size_t tc_extra_bytes(const v4moe_config& c, int64_t T);
 
+// Router GEMM: the reduction is split so that about this many CTAs run; the
+// workspace holds ksplit partial logit arrays [T, E].
+constexpr int kRouteTargetCtas = 148;
+int route_ksplit(const v4moe_config& c, int64_t T);
+
 // Shared expert on the token-major f16 GEMM (int8 weights widened to f16 in
 // the workspace) from this many tokens on.
 constexpr int kShMinTokens = 512;
@@ -40,7 +45,7 @@ DecodeBuffers dec_buffers(const v4moe_config& c, int64_t T);
 // Workspace carve-up for T tokens. All offsets are 256-byte aligned.
 struct WsLayout {
   size_t status = 0;        // uint32 status word + spare words (256 B)
-  size_t scores = 0;        // [T, E] fp32 router scores
+  size_t scores = 0;        // router: [ksplit, T, E] fp32 partial logits; decode: [T, E] scores
   size_t chunk_counts = 0;  // [nchunks, E] int32
   size_t chunk_base = 0;    // [nchunks, E] int32
   size_t h = 0;             // [T*k, I] bf16 routed intermediates (sorted order)
@@ -66,7 +71,7 @@ inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
     return o;
   };
   L.status = take(256);
-  L.scores = take(size_t(T) * c.n_experts * 4);
+  L.scores = take(size_t(route_ksplit(c, T)) * T * c.n_experts * 4);
   L.nchunks = int((S + kPermChunk - 1) / kPermChunk);
   if (L.nchunks < 1) L.nchunks = 1;
   L.chunk_counts = take(size_t(L.nchunks) * c.n_experts * 4);
@@ -89,9 +94,11 @@ inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
 
 // ---------------------------------------------------------------- launchers
 // Each returns cudaGetLastError() of its launches.
+// Router (any T): tcgen05 gate GEMM into the partial logits `part`, then the
+// per-token selection.
 cudaError_t launch_route(const v4moe_config& c, int T, const __nv_bfloat16* x,
                          const __nv_bfloat16* gate, const float* bias, const int32_t* token_ids,
-                         const int32_t* tid2eid, int32_t* topk_ids, float* topk_w, float* scores,
+                         const int32_t* tid2eid, int32_t* topk_ids, float* topk_w, float* part,
                          uint32_t* status, cudaStream_t st);
 
 cudaError_t launch_permute(const v4moe_config& c, int T, const int32_t* topk_ids, int32_t* counts,
