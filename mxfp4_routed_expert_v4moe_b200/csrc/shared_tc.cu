@@ -112,6 +112,49 @@ __device__ __forceinline__ void tma_load_3d_s(void* dst, const void* tmap, int x
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((max(-126, min(127, e)) + 127) << 23); }
 
+// One round of the combine (32 output rows from m0) for a warp's 32 tokens
+// (first token tq): lane l takes token 4 g + l / 8 and columns 4 (l % 8) .. + 3
+// for g = 0 .. 7, so a load instruction reads four tokens' 128-byte row
+// pieces; all of a token's NJ slot rows are in flight at once (slots that do
+// not exist read row 0 and are left out of the sum). wj / pj: this lane's
+// token's routing weights and slot positions; tb: the shared term of the
+// round, [token][column] with row stride kSXch.
+template <int NJ>
+__device__ __forceinline__ void combine_round(const ShParams& P, const float (&wj)[8], const int (&pj)[8],
+                                              const float* tb, int tq, int sl, int c4, int m0) {
+#pragma unroll 2
+  for (int g = 0; g < 8; ++g) {
+    const int tl = 4 * g + sl;  // token within the warp's 32
+    float w[NJ];
+    int p[NJ];
+    float4 y[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      w[j] = __shfl_sync(0xffffffffu, wj[j], tl);
+      p[j] = __shfl_sync(0xffffffffu, pj[j], tl);
+      y[j] = __ldg(reinterpret_cast<const float4*>(P.y_slot + size_t(max(p[j], 0)) * P.H + m0 + c4));
+    }
+    float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      if (p[j] >= 0) {
+        a.x = fmaf(w[j], y[j].x, a.x);
+        a.y = fmaf(w[j], y[j].y, a.y);
+        a.z = fmaf(w[j], y[j].z, a.z);
+        a.w = fmaf(w[j], y[j].w, a.w);
+      }
+    }
+    const int t2 = tq + tl;
+    if (t2 < P.T) {
+      const float* sp = tb + tl * kSXch + c4;
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x + sp[0], a.y + sp[1]);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(a.z + sp[2], a.w + sp[3]);
+      *reinterpret_cast<uint2*>(P.out + size_t(t2) * P.H + m0 + c4) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kSThreads, 1)
     k_sh_gemm(ShParams P, const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB) {
   extern __shared__ __align__(1024) char smem_raw[];
@@ -251,10 +294,9 @@ __global__ void __launch_bounds__(kSThreads, 1)
           }
         }
       } else {
-        // combine, 128 output rows in four rounds of 32. The shared term
-        // (thread = token) goes through this warp's transpose buffer; then
-        // lane l takes token 4 i + l / 8 and columns 4 (l % 8) .. + 3, so a
-        // load instruction reads four tokens' 128-byte row pieces.
+        // combine, 128 output rows in four rounds of 32: the shared term
+        // (thread = token) goes through this warp's transpose buffer, then
+        // combine_round adds the routed slots.
         float wj[8];
         int pj[8];
 #pragma unroll
@@ -286,39 +328,10 @@ __global__ void __launch_bounds__(kSThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) tb[lane * kSXch + i] = __uint_as_float(ra[i]) * __ldg(P.scale + m0 + i);
           __syncwarp();
-#pragma unroll 2
-          for (int g = 0; g < 8; ++g) {
-            const int tl = 4 * g + sl;  // token within the lane quarter
-            // all of the token's slot rows in flight at once: slots that do
-            // not exist read row 0 and are left out of the sum
-            float w[8];
-            int p[8];
-            float4 y[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              w[j] = __shfl_sync(0xffffffffu, wj[j], tl);
-              p[j] = __shfl_sync(0xffffffffu, pj[j], tl);
-              y[j] = __ldg(reinterpret_cast<const float4*>(P.y_slot + size_t(max(p[j], 0)) * P.H + m0 + c4));
-            }
-            float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (p[j] >= 0) {
-                a.x = fmaf(w[j], y[j].x, a.x);
-                a.y = fmaf(w[j], y[j].y, a.y);
-                a.z = fmaf(w[j], y[j].z, a.z);
-                a.w = fmaf(w[j], y[j].w, a.w);
-              }
-            }
-            const int t2 = t0 + 32 * q + tl;
-            if (t2 < P.T) {
-              const float* sp = tb + tl * kSXch + c4;
-              const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x + sp[0], a.y + sp[1]);
-              const __nv_bfloat162 hi = __floats2bfloat162_rn(a.z + sp[2], a.w + sp[3]);
-              *reinterpret_cast<uint2*>(P.out + size_t(t2) * P.H + m0 + c4) =
-                  make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
-            }
-          }
+          if (P.k <= 6)
+            combine_round<6>(P, wj, pj, tb, t0 + 32 * q, sl, c4, m0);
+          else
+            combine_round<8>(P, wj, pj, tb, t0 + 32 * q, sl, c4, m0);
           __syncwarp();
         }
       }
