@@ -185,6 +185,22 @@ int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const voi
                     int32_t* counts, int32_t* offsets, int32_t* sorted_slot, int32_t* slot_pos,
                     void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* W8A16 linear ("config.json" quantization_config, group "linears_w8a16":
+ * int8 weights, symmetric, one scale per output channel, 16-bit float
+ * activations; its targets are the attention projections fused_wqa_wkv,
+ * wq_b, wo_a, wo_b, the indexer's wq_b and compressor wkv, and the shared
+ * expert's gate_up_proj / down_proj):
+ *   out[t, n] = bf16( scale[n] * sum_k q[n, k] * x[t, k] ),  fp32 accumulation
+ *   x [T, K] bf16, q [N, K] int8 (row-major, 16-byte aligned), scale [N] fp32,
+ *   out [T, N] bf16 (16-byte aligned, may not alias x).
+ * Requirements: N % 32 == 0, K % 64 == 0. The weights are widened exactly to
+ * bf16 in the workspace (v4moe_linear_w8a16_workspace_bytes(T, N, K) bytes,
+ * 256-byte aligned; its first 256 bytes hold the device status word as for
+ * the other calls) and multiplied on the tensor cores. T == 0 is a no-op. */
+size_t v4moe_linear_w8a16_workspace_bytes(int32_t T, int32_t N, int32_t K);
+int32_t v4moe_linear_w8a16(int32_t T, int32_t N, int32_t K, const void* x, const int8_t* q,
+                           const float* scale, void* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, reads the device status word of `ws` and returns
  * V4MOE_OK, V4MOE_ERR_DATA or V4MOE_ERR_TIMEOUT (or V4MOE_ERR_LAUNCH if the
  * copy fails). Test/debug only. */

@@ -29,7 +29,8 @@ V4MOE_ERR_TIMEOUT = 6
 EXPORTED = ("v4moe_workspace_bytes", "v4moe_route", "v4moe_permute", "v4moe_forward",
             "v4moe_read_device_status", "v4moe_clear_device_status", "v4moe_status_string",
             "v4moe_profile_enable", "v4moe_profile_reset", "v4moe_profile_read",
-            "v4moe_launch_count", "v4moe_permute_static", "v4moe_layer")
+            "v4moe_launch_count", "v4moe_permute_static", "v4moe_layer",
+            "v4moe_linear_w8a16_workspace_bytes", "v4moe_linear_w8a16")
 
 
 class V4moeError(RuntimeError):
@@ -80,6 +81,10 @@ def load(path: str | None = None):
             L.v4moe_layer.argtypes = [cfgp, i32, P, P, P, P, P, ctypes.POINTER(v4moe_weights), P, P, P, P,
                                       P, P, P, P, sz, P]
             L.v4moe_layer.restype = i32
+            L.v4moe_linear_w8a16_workspace_bytes.argtypes = [i32, i32, i32]
+            L.v4moe_linear_w8a16_workspace_bytes.restype = sz
+            L.v4moe_linear_w8a16.argtypes = [i32, i32, i32, P, P, P, P, P, sz, P]
+            L.v4moe_linear_w8a16.restype = i32
             L.v4moe_read_device_status.argtypes = [P, P]
             L.v4moe_read_device_status.restype = i32
             L.v4moe_clear_device_status.argtypes = [P, P]
@@ -178,6 +183,15 @@ def v4moe_layer(cfg, T, x, gate, bias, token_ids, tid2eid, weights, topk_ids, to
                               _ptr(tid2eid), ctypes.byref(weights), _ptr(topk_ids), _ptr(topk_w),
                               _ptr(counts), _ptr(offsets), _ptr(sorted_slot), _ptr(slot_pos),
                               _ptr(out), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def v4moe_linear_w8a16_workspace_bytes(T: int, N: int, K: int) -> int:
+    return load().v4moe_linear_w8a16_workspace_bytes(T, N, K)
+
+
+def v4moe_linear_w8a16(T, N, K, x, q, scale, out, ws, ws_bytes, stream=None) -> int:
+    return load().v4moe_linear_w8a16(T, N, K, _ptr(x), _ptr(q), _ptr(scale), _ptr(out), _ptr(ws), ws_bytes,
+                                     _stream(stream))
 
 
 def v4moe_read_device_status(ws, stream=None) -> int:

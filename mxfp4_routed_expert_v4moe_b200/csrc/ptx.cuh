@@ -270,6 +270,11 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
+// The same with bf16 A and B (formats 1).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return idesc_f16_f32(M, N) | (1u << 7) | (1u << 10);
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -52,11 +52,6 @@ __device__ __forceinline__ bool rwait(uint64_t* bar, uint32_t parity, volatile i
   return false;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A and B (formats 1), fp32 D.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-  return idesc_f16_f32(M, N) | (1u << 7) | (1u << 10);
-}
-
 // grid (token tiles, K splits, expert tiles); box_n: gate rows per TMA box.
 __global__ void __launch_bounds__(kRThreads, 1)
     k_route_gemm(int T, int E, int nk, int nk_per, int box_n, float* __restrict__ part, uint32_t* status,

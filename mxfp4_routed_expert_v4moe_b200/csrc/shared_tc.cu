@@ -61,7 +61,7 @@ constexpr int kSSmem = kSOffBar + 256 + 1024;
 static_assert(kSSmem <= 232448, "dynamic shared memory per block");
 constexpr uint32_t kSTries = 1u << 21;
 
-enum { kSW13 = 0, kSW2 = 1 };
+enum { kSW13 = 0, kSW2 = 1, kSLin = 2 };
 
 struct SBars {
   uint64_t full[kSStages];
@@ -88,7 +88,8 @@ struct ShParams {
   const float* topk_w;
   const int32_t* slot_pos;
   const float* y_slot;   // [T k, H] routed outputs in slot order
-  __nv_bfloat16* out;    // [T, H]
+  __nv_bfloat16* out;    // [T, H]; linear mode: [T, N]
+  int N;                 // linear mode: output channels
   uint32_t* status;
 };
 
@@ -163,6 +164,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
   volatile int* abort_flag = &B.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool w13 = P.mode == kSW13;
+  const bool lin = P.mode == kSLin;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSStages; ++s) {
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     uint32_t gc = 0, lt = 0;
     bool ok = true;
-    const uint32_t idesc = idesc_f16_f32(SMt, SNr);
+    const uint32_t idesc = lin ? idesc_bf16_f32(SMt, SNr) : idesc_f16_f32(SMt, SNr);
     for (int ti = blockIdx.x; ti < P.ntiles && ok; ti += gridDim.x, ++lt) {
       const uint32_t b = lt & 1u, v = lt >> 1;
       if (!swait(&B.acc_empty[b], (v & 1u) ^ 1u, abort_flag, P.status)) break;
@@ -258,6 +260,36 @@ __global__ void __launch_bounds__(kSThreads, 1)
       if (!__all_sync(0xffffffffu, swait(&B.acc_full[b], v & 1u, abort_flag, P.status)) || *abort_flag) break;
       tc_fence_after();
       const uint32_t acc = tmem + b * SNr + (uint32_t(32 * q) << 16);
+      if (lin) {
+        // out[t, n] = bf16(scale[n] * acc), 128 channels per warp in rounds of 32
+        const int t = t0 + 32 * q + lane;
+#pragma unroll 1
+        for (int r = 0; r < 4; ++r) {
+          const int cc = 128 * half + 32 * r;
+          uint32_t ra[32];
+          tmem_ld_32x32b_x32(acc + cc, ra);
+          tmem_wait_ld();
+          if (r == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B.acc_empty[b]);
+          }
+          const int n0 = rb * SNr + cc;
+          if (t < P.T && n0 < P.N) {  // N % 32 == 0: a round is all in or all out
+            uint32_t o[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(ra[i]) * __ldg(P.scale + n0 + i),
+                                                             __uint_as_float(ra[i + 1]) * __ldg(P.scale + n0 + i + 1));
+              o[i >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(P.out + size_t(t) * P.N + n0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+        }
+        continue;
+      }
       const int tok = t0 + 32 * q + lane;
       const bool valid = tok < P.T;
       if (w13) {
@@ -377,6 +409,28 @@ __global__ void __launch_bounds__(256) k_s8_to_f16(const int8_t* __restrict__ a,
   }
 }
 
+// int8 -> bf16, exact (|q| <= 128 has at most 8 significant bits): the fp32
+// value's upper 16 bits. n % 16 == 0, both pointers 16-byte aligned.
+__global__ void __launch_bounds__(256) k_s8_to_bf16(const int8_t* __restrict__ q, __nv_bfloat16* __restrict__ w,
+                                                    size_t n) {
+  const size_t n16 = n / 16;
+  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n16; i += size_t(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(q) + i);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int b0 = int(int8_t(in[j] & 0xFFu)), b1 = int(int8_t((in[j] >> 8) & 0xFFu));
+      const int b2 = int(int8_t((in[j] >> 16) & 0xFFu)), b3 = int(int8_t(in[j] >> 24));
+      o[2 * j] = (__float_as_uint(float(b0)) >> 16) | (__float_as_uint(float(b1)) & 0xFFFF0000u);
+      o[2 * j + 1] = (__float_as_uint(float(b2)) >> 16) | (__float_as_uint(float(b3)) & 0xFFFF0000u);
+    }
+    uint4* d = reinterpret_cast<uint4*>(w) + 2 * i;
+    d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 sh_encode_fn() {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -390,9 +444,10 @@ PFN_cuTensorMapEncodeTiled_v12000 sh_encode_fn() {
   return fn;
 }
 
-// f16 maps, 128-byte swizzle, box of 64 elements (128 B) along K.
-// 2-D: [rows][cols]; 3-D: [2][rows][cols] (gate half, up half).
-bool sh_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t halves, uint32_t box_rows) {
+// 16-bit maps (f16 unless given), 128-byte swizzle, box of 64 elements (128 B)
+// along K. 2-D: [rows][cols]; 3-D: [2][rows][cols] (gate half, up half).
+bool sh_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t halves, uint32_t box_rows,
+            CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16) {
   auto fn = sh_encode_fn();
   if (!fn) return false;
   if (rows == 0) rows = 1;
@@ -400,7 +455,7 @@ bool sh_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint
   const cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
   const cuuint32_t box[3] = {uint32_t(SKc), box_rows, uint32_t(halves)};
   const cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, halves > 1 ? 3 : 2, const_cast<void*>(base), dims, strides, box, es,
+  return fn(m, dt, halves > 1 ? 3 : 2, const_cast<void*>(base), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -487,6 +542,34 @@ cudaError_t launch_sh_w2_combine(const ForwardArgs& a, char* extra, cudaStream_t
   P.scale = a.w.sh_w2_scale;
   return launch_kernel("sh_w2", k_sh_gemm, dim3(std::min(sm_count(), P.ntiles)), dim3(kSThreads), kSSmem, st, true,
                        P, mA, mB);
+}
+
+size_t linear_w8a16_ws_bytes(int64_t N, int64_t K) { return 256 + align_up(size_t(N) * K * 2); }
+
+cudaError_t launch_linear_w8a16(int T, int N, int K, const __nv_bfloat16* x, const int8_t* q, const float* scale,
+                                __nv_bfloat16* out, char* ws, cudaStream_t st) {
+  __nv_bfloat16* qw = reinterpret_cast<__nv_bfloat16*>(ws + 256);
+  const int sms = sm_count();
+  cudaError_t e = launch_kernel("lin_widen", k_s8_to_bf16, dim3(4 * sms), dim3(256), 0, st, false, q, qw,
+                                size_t(N) * K);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mA, mB;
+  constexpr auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!sh_map(&mA, x, K, T, 1, SMt, BF) || !sh_map(&mB, qw, K, N, 1, SNr, BF)) return cudaErrorInvalidValue;
+  set_smem(k_sh_gemm, kSSmem);
+  ShParams P = {};
+  P.T = T;
+  P.H = 0;
+  P.N = N;
+  P.mode = kSLin;
+  P.nb = (N + SNr - 1) / SNr;
+  P.ntiles = (T + SMt - 1) / SMt * P.nb;
+  P.nk = K / SKc;
+  P.scale = scale;
+  P.out = out;
+  P.status = reinterpret_cast<uint32_t*>(ws);
+  return launch_kernel("lin_gemm", k_sh_gemm, dim3(std::min(sms, P.ntiles)), dim3(kSThreads), kSSmem, st, true, P,
+                       mA, mB);
 }
 
 }  // namespace v4moe

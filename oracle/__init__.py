@@ -56,6 +56,9 @@ def lib():
         if _lib is None:
             L = ctypes.CDLL(build())
             P, i32, d = ctypes.c_void_p, ctypes.c_int32, ctypes.c_double
+            L.orc_linear_w8a16.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+            L.orc_linear_w8a16.restype = None
             L.orc_bf16_to_double.argtypes = [ctypes.c_uint16]
             L.orc_bf16_to_double.restype = d
             L.orc_e2m1.argtypes = [ctypes.c_int]
@@ -205,3 +208,17 @@ def permute(ids: np.ndarray, E: int):
     if rc:
         raise ValueError("out-of-range expert id")
     return counts, offsets, sorted_slot, slot_pos
+
+
+def linear_w8a16(x_bf16: np.ndarray, q: np.ndarray, scale: np.ndarray, rows=None) -> np.ndarray:
+    """W8A16 linear (config group linears_w8a16): out[t, n] = sum_k x[t, k] q[n, k]
+    scale[n] in fp64. x_bf16: [T, K] uint16 bf16 bit patterns; q: [N, K] int8;
+    scale: [N] fp32. rows: optional token subset (the rows of out returned)."""
+    x = np.ascontiguousarray(x_bf16 if rows is None else x_bf16[np.asarray(rows)], np.uint16)
+    q = np.ascontiguousarray(q, np.int8)
+    scale = np.ascontiguousarray(scale, np.float32)
+    T, K = x.shape
+    N = q.shape[0]
+    out = np.zeros((T, N), np.float64)
+    lib().orc_linear_w8a16(T, N, K, _p(x), _p(q), _p(scale), _p(out))
+    return out

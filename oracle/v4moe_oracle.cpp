@@ -365,4 +365,20 @@ int orc_moe_dense(const OrcLayer* L, const int32_t* ids, const double* w, double
   return 0;
 }
 
+// [P5] quantization_config, group linears_w8a16 (weights: 8-bit int,
+// symmetric, strategy channel; input activations: 16-bit float; targets the
+// attention projections and the shared expert's two projections): the
+// dequantised weight is q[n, k] * scale[n], and the linear is
+//   out[t, n] = sum_k x[t, k] * q[n, k] * scale[n]     (fp64, bf16 x exact).
+void orc_linear_w8a16(int32_t T, int32_t N, int32_t K, const uint16_t* x, const int8_t* q, const float* scale,
+                      double* out) {
+  for (int t = 0; t < T; ++t)
+    for (int n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int k = 0; k < K; ++k)
+        acc += orc_bf16_to_double(x[int64_t(t) * K + k]) * (double(q[int64_t(n) * K + k]) * double(scale[n]));
+      out[int64_t(t) * N + n] = acc;
+    }
+}
+
 }  // extern "C"

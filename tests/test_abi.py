@@ -79,3 +79,15 @@ def test_invalid_arguments_rejected_before_launch(lib):
 def test_python_binding_has_the_c_names():
     for s in declared_symbols():
         assert callable(getattr(V, s)), s
+
+
+def test_linear_w8a16_rejects_bad_shapes_before_any_launch():
+    import mxfp4_routed_expert_v4moe_b200 as V
+    assert V.v4moe_linear_w8a16_workspace_bytes(4, 64, 128) == 256 + 64 * 128 * 2
+    assert V.v4moe_linear_w8a16_workspace_bytes(4, 0, 128) == 0
+    # N % 32, K % 64, misaligned pointers: refused on the host
+    assert V.v4moe_linear_w8a16(4, 48, 128, 16, 16, 16, 32, 256, 1 << 20, 0) == V.V4MOE_ERR_INVALID_ARG
+    assert V.v4moe_linear_w8a16(4, 64, 96, 16, 16, 16, 32, 256, 1 << 20, 0) == V.V4MOE_ERR_INVALID_ARG
+    assert V.v4moe_linear_w8a16(4, 64, 128, 16, 8, 16, 32, 256, 1 << 20, 0) == V.V4MOE_ERR_INVALID_ARG
+    assert V.v4moe_linear_w8a16(4, 64, 128, 16, 16, 16, 32, 256, 100, 0) == V.V4MOE_ERR_WORKSPACE
+

@@ -329,3 +329,35 @@ def test_threaded_token_split_changes_nothing():
     assert np.array_equal(a, b)
     a2, h2, hs2 = lay.moe_tokens(np.array([6, 1]), ids, w, threads=2, want_h=True)
     assert np.array_equal(a2, a[[6, 1]])
+
+
+# ----------------------------------------------------------------------------- W8A16 linear
+
+def test_linear_w8a16_hand_case():
+    # x = [1, 2], q = [[1, 2], [3, -4]], scale = [0.5, 2]: (1 + 4) * 0.5 and (3 - 8) * 2
+    x = np.array([[0x3F80, 0x4000]], np.uint16)
+    q = np.array([[1, 2], [3, -4]], np.int8)
+    s = np.array([0.5, 2.0], np.float32)
+    assert O.linear_w8a16(x, q, s).tolist() == [[2.5, -10.0]]
+
+
+def test_linear_w8a16_scaled_identity_is_exact():
+    # q = c * I with scale 2^-3: out = x * c / 8 exactly (powers of two, small c)
+    K = 64
+    x = bf16(np.linspace(-3.0, 3.0, 2 * K).reshape(2, K))
+    for c in (-127, -3, 1, 5, 127):
+        q = (np.eye(K) * c).astype(np.int8)
+        s = np.full(K, 0.125, np.float32)
+        assert np.array_equal(O.linear_w8a16(x, q, s), bf16_val(x) * c * 0.125)
+
+
+def test_linear_w8a16_matches_numpy_and_row_subset():
+    rng = np.random.default_rng(3)
+    T, N, K = 5, 40, 96
+    x = bf16(rng.standard_normal((T, K)))
+    q = rng.integers(-127, 128, size=(N, K)).astype(np.int8)
+    s = (rng.random(N) * 0.01).astype(np.float32)
+    ref = bf16_val(x) @ (q.astype(np.float64) * s.astype(np.float64)[:, None]).T
+    got = O.linear_w8a16(x, q, s)
+    assert np.allclose(got, ref, rtol=1e-13, atol=1e-15)
+    assert np.array_equal(O.linear_w8a16(x, q, s, rows=[4, 1]), got[[4, 1]])
