@@ -33,6 +33,25 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s"
+LINEAR_METRIC = "W8A16 linear tokens/s"
+
+# W8A16 linear workloads: the linears_w8a16 targets of the config's attention
+# at prefill size, name -> (T tokens, G groups, N outputs per group, K inputs
+# per group). Shapes read from the config: fused_wqa_wkv q_lora_rank +
+# head_dim from hidden_size; wq_b num_attention_heads * head_dim from
+# q_lora_rank; wo_a o_groups groups of o_lora_rank from the group's heads *
+# head_dim; wo_b hidden_size from o_groups * o_lora_rank; the indexer's wq_b
+# index_n_heads * index_head_dim from q_lora_rank; the indexer compressor's wkv
+# index_head_dim from hidden_size (its width is not printed: the plainest
+# reading).
+LINEAR_WORKLOADS = {
+    "linear_fused_wqa_wkv_4096": (4096, 1, 1024 + 512, 4096),
+    "linear_wq_b_4096": (4096, 1, 64 * 512, 1024),
+    "linear_wo_a_4096": (4096, 8, 1024, 64 * 512 // 8),
+    "linear_wo_b_4096": (4096, 1, 4096, 8 * 1024),
+    "linear_indexer_wq_b_4096": (4096, 1, 64 * 128, 1024),
+    "linear_indexer_wkv_4096": (4096, 1, 128, 4096),
+}
 L2_FLUSH_BYTES = 512 << 20
 L2_CLEAN_BYTES = 256 << 20
 
@@ -231,6 +250,32 @@ def oracle_sample(wl, li, n_tok, seconds):
 
 # ----------------------------------------------------------------------------- main
 
+def run_reference_linear(args):
+    import inputs as IN
+    import oracle as O
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    T, G, N, K = LINEAR_WORKLOADS[args.workload]
+    x_bits = IN.normal_bf16(0, 1, T * G * K).reshape(T, G * K)
+    q, sc = IN.int8_normal(0, 2, G * N, K, 0.02)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        O.linear_w8a16_grouped(x_bits, q, sc, G, rows=[0])
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    ms = 1e3 * float(np.mean(times))
+    value = 1 / (ms / 1e3)
+    print(json.dumps({"impl": "reference", "metric": LINEAR_METRIC, "value": value, "unit": "tokens/s",
+                      "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic", "config": {"workload": args.workload, "T": T, "G": G, "N": N, "K": K},
+                      "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                       "sample": f"1 token row of {args.workload} per step"},
+                      "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                              "d2h_bytes_per_step": 0}}), flush=True)
+
+
 def run_reference(args):
     import inputs as IN
     rank = int(os.environ.get("RANK", "0"))
@@ -260,8 +305,114 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_linear(args):
+    """One W8A16 linear call per step (v4moe_linear_w8a16), same timing rules."""
+    import torch
+
+    import inputs as IN
+    import mxfp4_routed_expert_v4moe_b200 as V
+    T, G, N, K = LINEAR_WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    x_bits = IN.normal_bf16(0, 1, T * G * K).reshape(T, G * K)
+    q, sc = IN.int8_normal(0, 2, G * N, K, 0.02)
+    x = torch.from_numpy(x_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    qd, sd = torch.from_numpy(q).to(dev), torch.from_numpy(sc).to(dev)
+    out = torch.empty((T, G * N), dtype=torch.bfloat16, device=dev)
+    nb = V.v4moe_linear_w8a16_grouped_workspace_bytes(T, G, N, K)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.ones(L2_CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)
+        clean.sum()
+
+    def step(xx=x, oo=out):
+        V.check(V.v4moe_linear_w8a16_grouped(T, G, N, K, xx, qd, sd, oo, ws, nb), "v4moe_linear_w8a16_grouped")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
+    clocks.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches0 = V.v4moe_launch_count()
+    for i in range(args.steps):
+        flush_l2(i)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    launches = V.v4moe_launch_count() - launches0
+    ms_step = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_host = torch.empty((T, G * N), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush_l2(i)
+        e2e_evs[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        out_host.copy_(out, non_blocking=True)
+        e2e_evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs) / args.steps
+    clk = clocks.stop()
+    V.v4moe_profile_reset()
+    V.v4moe_profile_enable(True)
+    for i in range(args.steps):
+        flush_l2(i)
+        step()
+    torch.cuda.synchronize(dev)
+    prof = V.v4moe_profile_read()
+    V.v4moe_profile_enable(False)
+    pk = peaks()
+    flops = 2.0 * T * G * N * K
+    gemm_ms = prof.get("lin_gemm", (0.0, 1))[0] / max(prof.get("lin_gemm", (0.0, 1))[1], 1)
+    achieved = flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
+    lin_bytes = G * (N * K + 4 * N + 2 * T * K + 2 * T * N)
+    line = {"metric": LINEAR_METRIC, "value": T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "T": T, "G": G, "N": N, "K": K,
+                       "weights": "int8 per output channel + fp32 scales", "parallelism": f"replicas{world}",
+                       "l2": "flushed between timed steps (512 MiB write, then 256 MiB read)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16"], "peak_src": pk["src"], "kernel": "lin_gemm",
+                         "kernel_ms": gemm_ms, "algorithmic_per_launch": flops, "traffic": None},
+            "layer_roofline": {"algorithmic_flops": flops, "algorithmic_bytes": lin_bytes,
+                               "roofline_ms": max(flops / (pk["bf16"] * 1e12), lin_bytes / (pk["hbm"] * 1e9)) * 1e3},
+            "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches_per_step": v[1] / args.steps}
+                        for k, v in sorted(prof.items(), key=lambda kv: -kv[1][0])},
+            "e2e": {"value": T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(T * G * K * 2),
+                    "d2h_bytes_per_step": int(T * G * N * 2)},
+            "gpu_launches": int(launches), "clocks": clk}
+    line["layer_roofline"]["frac"] = line["layer_roofline"]["roofline_ms"] / ms_step
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle as O
+        rows, reps, t0 = [0, 1], 0, time.perf_counter()
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            O.linear_w8a16_grouped(x_bits, q, sc, G, rows=rows)
+            reps += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": reps * len(rows) / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{reps} x {len(rows)} token rows of {args.workload}, {el:.1f} s single-threaded fp64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.workload in LINEAR_WORKLOADS:
+        if args.impl == "reference":
+            return run_reference_linear(args)
+        return run_linear(args)
     if args.impl == "reference":
         return run_reference(args)
     import torch

@@ -201,6 +201,20 @@ size_t v4moe_linear_w8a16_workspace_bytes(int32_t T, int32_t N, int32_t K);
 int32_t v4moe_linear_w8a16(int32_t T, int32_t N, int32_t K, const void* x, const int8_t* q,
                            const float* scale, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* The same linear in G independent groups (the config's wo_a: o_groups = 8
+ * groups of heads, each projected by its own o_lora_rank x (heads per group *
+ * head_dim) block of one weight matrix):
+ *   out[t, g N + n] = bf16( scale[g N + n] * sum_k q[g N + n, k] * x[t, g K + k] )
+ *   x [T, G K] bf16, q [G N, K] int8, scale [G N] fp32, out [T, G N] bf16,
+ * alignment and requirements as above (N % 32 == 0, K % 64 == 0, G >= 1;
+ * G N and G K at most 2^30); workspace
+ * v4moe_linear_w8a16_grouped_workspace_bytes(T, G, N, K) bytes. G == 1 is
+ * v4moe_linear_w8a16. */
+size_t v4moe_linear_w8a16_grouped_workspace_bytes(int32_t T, int32_t G, int32_t N, int32_t K);
+int32_t v4moe_linear_w8a16_grouped(int32_t T, int32_t G, int32_t N, int32_t K, const void* x,
+                                   const int8_t* q, const float* scale, void* out, void* ws,
+                                   size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, reads the device status word of `ws` and returns
  * V4MOE_OK, V4MOE_ERR_DATA or V4MOE_ERR_TIMEOUT (or V4MOE_ERR_LAUNCH if the
  * copy fails). Test/debug only. */

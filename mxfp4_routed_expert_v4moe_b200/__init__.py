@@ -30,7 +30,8 @@ EXPORTED = ("v4moe_workspace_bytes", "v4moe_route", "v4moe_permute", "v4moe_forw
             "v4moe_read_device_status", "v4moe_clear_device_status", "v4moe_status_string",
             "v4moe_profile_enable", "v4moe_profile_reset", "v4moe_profile_read",
             "v4moe_launch_count", "v4moe_permute_static", "v4moe_layer",
-            "v4moe_linear_w8a16_workspace_bytes", "v4moe_linear_w8a16")
+            "v4moe_linear_w8a16_workspace_bytes", "v4moe_linear_w8a16",
+            "v4moe_linear_w8a16_grouped_workspace_bytes", "v4moe_linear_w8a16_grouped")
 
 
 class V4moeError(RuntimeError):
@@ -85,6 +86,10 @@ def load(path: str | None = None):
             L.v4moe_linear_w8a16_workspace_bytes.restype = sz
             L.v4moe_linear_w8a16.argtypes = [i32, i32, i32, P, P, P, P, P, sz, P]
             L.v4moe_linear_w8a16.restype = i32
+            L.v4moe_linear_w8a16_grouped_workspace_bytes.argtypes = [i32, i32, i32, i32]
+            L.v4moe_linear_w8a16_grouped_workspace_bytes.restype = sz
+            L.v4moe_linear_w8a16_grouped.argtypes = [i32, i32, i32, i32, P, P, P, P, P, sz, P]
+            L.v4moe_linear_w8a16_grouped.restype = i32
             L.v4moe_read_device_status.argtypes = [P, P]
             L.v4moe_read_device_status.restype = i32
             L.v4moe_clear_device_status.argtypes = [P, P]
@@ -192,6 +197,15 @@ def v4moe_linear_w8a16_workspace_bytes(T: int, N: int, K: int) -> int:
 def v4moe_linear_w8a16(T, N, K, x, q, scale, out, ws, ws_bytes, stream=None) -> int:
     return load().v4moe_linear_w8a16(T, N, K, _ptr(x), _ptr(q), _ptr(scale), _ptr(out), _ptr(ws), ws_bytes,
                                      _stream(stream))
+
+
+def v4moe_linear_w8a16_grouped_workspace_bytes(T: int, G: int, N: int, K: int) -> int:
+    return load().v4moe_linear_w8a16_grouped_workspace_bytes(T, G, N, K)
+
+
+def v4moe_linear_w8a16_grouped(T, G, N, K, x, q, scale, out, ws, ws_bytes, stream=None) -> int:
+    return load().v4moe_linear_w8a16_grouped(T, G, N, K, _ptr(x), _ptr(q), _ptr(scale), _ptr(out), _ptr(ws),
+                                             ws_bytes, _stream(stream))
 
 
 def v4moe_read_device_status(ws, stream=None) -> int:

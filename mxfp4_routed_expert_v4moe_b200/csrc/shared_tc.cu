@@ -35,6 +35,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "launch.cuh"
@@ -88,10 +89,25 @@ struct ShParams {
   const float* topk_w;
   const int32_t* slot_pos;
   const float* y_slot;   // [T k, H] routed outputs in slot order
-  __nv_bfloat16* out;    // [T, H]; linear mode: [T, N]
-  int N;                 // linear mode: output channels
+  __nv_bfloat16* out;    // [T, H]; linear mode: [T, G N]
+  // linear mode: G groups of N output channels over K inputs each (group g
+  // reads x columns g K .. and weight rows g N ..); bn weight rows per tile
+  // (128 or 256, nbg blocks per group); order 1 walks the token tiles of a
+  // weight block before the next block (mt token tiles).
+  int G, N, K, bn, nbg, mt, order;
   uint32_t* status;
 };
+
+// Tile ti -> first token, weight-row block (over all groups in linear mode).
+__device__ __forceinline__ void tile_of(const ShParams& P, int ti, int& t0, int& rb) {
+  if (P.order) {
+    rb = ti / P.mt;
+    t0 = (ti - rb * P.mt) * SMt;
+  } else {
+    t0 = (ti / P.nb) * SMt;
+    rb = ti % P.nb;
+  }
+}
 
 __device__ __forceinline__ bool swait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status) {
   for (uint32_t i = 0; i < kSTries; ++i) {
@@ -195,8 +211,13 @@ __global__ void __launch_bounds__(kSThreads, 1)
     prefetch_tmap(&tmB);
     uint32_t gc = 0;
     bool ok = true;
+    const uint32_t stage_bytes = uint32_t(kSA + (lin ? P.bn : SNr) * SKc * 2);
     for (int ti = blockIdx.x; ti < P.ntiles && ok; ti += gridDim.x) {
-      const int t0 = (ti / P.nb) * SMt, rb = ti % P.nb;
+      int t0, rb;
+      tile_of(P, ti, t0, rb);
+      const int g = lin ? rb / P.nbg : 0;
+      const int acol = lin ? g * P.K : 0;
+      const int brow = lin ? g * P.N + (rb - g * P.nbg) * P.bn : rb * SNr;
       for (int c = 0; c < P.nk; ++c, ++gc) {
         const int s = gc % kSStages;
         const uint32_t u = gc / kSStages;
@@ -205,12 +226,12 @@ __global__ void __launch_bounds__(kSThreads, 1)
           break;
         }
         char* st = smem + s * kSStage;
-        mbar_arrive_expect_tx(&B.full[s], uint32_t(kSStage));
-        tma_load_2d(st, &tmA, c * SKc, t0, &B.full[s]);
+        mbar_arrive_expect_tx(&B.full[s], stage_bytes);
+        tma_load_2d(st, &tmA, acol + c * SKc, t0, &B.full[s]);
         if (w13)  // 128 gate rows, then the matching 128 up rows
           tma_load_3d_s(st + kSA, &tmB, c * SKc, rb * (SNr / 2), 0, &B.full[s]);
         else
-          tma_load_2d(st + kSA, &tmB, c * SKc, rb * SNr, &B.full[s]);
+          tma_load_2d(st + kSA, &tmB, c * SKc, brow, &B.full[s]);
       }
     }
     // nothing may still be landing in shared memory when the CTA exits
@@ -222,7 +243,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     uint32_t gc = 0, lt = 0;
     bool ok = true;
-    const uint32_t idesc = lin ? idesc_bf16_f32(SMt, SNr) : idesc_f16_f32(SMt, SNr);
+    const uint32_t idesc = lin ? idesc_bf16_f32(SMt, P.bn) : idesc_f16_f32(SMt, SNr);
     for (int ti = blockIdx.x; ti < P.ntiles && ok; ti += gridDim.x, ++lt) {
       const uint32_t b = lt & 1u, v = lt >> 1;
       if (!swait(&B.acc_empty[b], (v & 1u) ^ 1u, abort_flag, P.status)) break;
@@ -256,26 +277,32 @@ __global__ void __launch_bounds__(kSThreads, 1)
     uint32_t lt = 0;
     for (int ti = blockIdx.x; ti < P.ntiles; ti += gridDim.x, ++lt) {
       const uint32_t b = lt & 1u, v = lt >> 1;
-      const int t0 = (ti / P.nb) * SMt, rb = ti % P.nb;
+      int t0, rb;
+      tile_of(P, ti, t0, rb);
       if (!__all_sync(0xffffffffu, swait(&B.acc_full[b], v & 1u, abort_flag, P.status)) || *abort_flag) break;
       tc_fence_after();
       const uint32_t acc = tmem + b * SNr + (uint32_t(32 * q) << 16);
       if (lin) {
-        // out[t, n] = bf16(scale[n] * acc), 128 channels per warp in rounds of 32
+        // out[t, g N + n] = bf16(scale[g N + n] * acc): bn / 2 channels per
+        // warp in rounds of 32
         const int t = t0 + 32 * q + lane;
+        const int g = rb / P.nbg;
+        const int nrounds = P.bn / 64;
+        const size_t ld = size_t(P.G) * P.N;
 #pragma unroll 1
-        for (int r = 0; r < 4; ++r) {
-          const int cc = 128 * half + 32 * r;
+        for (int r = 0; r < nrounds; ++r) {
+          const int cc = (P.bn / 2) * half + 32 * r;
           uint32_t ra[32];
           tmem_ld_32x32b_x32(acc + cc, ra);
           tmem_wait_ld();
-          if (r == 3) {
+          if (r == nrounds - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&B.acc_empty[b]);
           }
-          const int n0 = rb * SNr + cc;
-          if (t < P.T && n0 < P.N) {  // N % 32 == 0: a round is all in or all out
+          const int nl = (rb - g * P.nbg) * P.bn + cc;  // channel within the group
+          if (t < P.T && nl < P.N) {  // N % 32 == 0: a round is all in or all out
+            const int n0 = g * P.N + nl;
             uint32_t o[16];
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
@@ -283,7 +310,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
                                                              __uint_as_float(ra[i + 1]) * __ldg(P.scale + n0 + i + 1));
               o[i >> 1] = *reinterpret_cast<const uint32_t*>(&h);
             }
-            uint4* dst = reinterpret_cast<uint4*>(P.out + size_t(t) * P.N + n0);
+            uint4* dst = reinterpret_cast<uint4*>(P.out + size_t(t) * ld + n0);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
           }
@@ -477,7 +504,7 @@ namespace {
 
 ShParams sh_params(const ForwardArgs& a, const int* sigma) {
   const v4moe_config& c = a.c;
-  ShParams P;
+  ShParams P = {};
   P.T = a.T;
   P.H = c.hidden;
   P.Is = c.shared_inter;
@@ -544,30 +571,58 @@ cudaError_t launch_sh_w2_combine(const ForwardArgs& a, char* extra, cudaStream_t
                        P, mA, mB);
 }
 
-size_t linear_w8a16_ws_bytes(int64_t N, int64_t K) { return 256 + align_up(size_t(N) * K * 2); }
+size_t linear_w8a16_ws_bytes(int64_t G, int64_t N, int64_t K) { return 256 + align_up(size_t(G) * N * K * 2); }
 
-cudaError_t launch_linear_w8a16(int T, int N, int K, const __nv_bfloat16* x, const int8_t* q, const float* scale,
-                                __nv_bfloat16* out, char* ws, cudaStream_t st) {
+namespace {
+
+// Weight rows per tile: 256 unless 128-row tiles fill the SMs' waves much
+// better. A 128-row tile moves 4/3 the operand bytes per flop of a 256-row
+// one and the GEMM is bound by that shared-memory fill rate: measured on B200
+// (4096 x 1536 x 4096: 2 waves of 256-row tiles 0.060 ms, 3 waves of 128-row
+// tiles 0.074 ms), a 128-row tile does ~0.6 of the work per unit time.
+int lin_block_rows(int mt, int G, int N, int sms) {
+  auto eff = [&](int bn) {
+    const int nbg = (N + bn - 1) / bn;
+    const double tiles = double(mt) * G * nbg;
+    const double waves = std::ceil(tiles / sms);
+    return tiles / (waves * sms) * double(N) / (double(nbg) * bn);
+  };
+  return eff(128) * 0.6 > eff(256) ? 128 : 256;
+}
+
+}  // namespace
+
+cudaError_t launch_linear_w8a16(int T, int G, int N, int K, const __nv_bfloat16* x, const int8_t* q,
+                                const float* scale, __nv_bfloat16* out, char* ws, cudaStream_t st) {
   __nv_bfloat16* qw = reinterpret_cast<__nv_bfloat16*>(ws + 256);
   const int sms = sm_count();
   cudaError_t e = launch_kernel("lin_widen", k_s8_to_bf16, dim3(4 * sms), dim3(256), 0, st, false, q, qw,
-                                size_t(N) * K);
+                                size_t(G) * N * K);
   if (e != cudaSuccess) return e;
-  CUtensorMap mA, mB;
-  constexpr auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!sh_map(&mA, x, K, T, 1, SMt, BF) || !sh_map(&mB, qw, K, N, 1, SNr, BF)) return cudaErrorInvalidValue;
-  set_smem(k_sh_gemm, kSSmem);
   ShParams P = {};
   P.T = T;
   P.H = 0;
+  P.G = G;
   P.N = N;
+  P.K = K;
   P.mode = kSLin;
-  P.nb = (N + SNr - 1) / SNr;
-  P.ntiles = (T + SMt - 1) / SMt * P.nb;
+  P.mt = (T + SMt - 1) / SMt;
+  P.bn = lin_block_rows(P.mt, G, N, sms);
+  P.nbg = (N + P.bn - 1) / P.bn;
+  P.nb = G * P.nbg;
+  P.ntiles = P.mt * P.nb;
+  // the operand with more bytes is read once: walk the token tiles of a weight
+  // block first when the weights are the larger operand
+  P.order = N > T ? 1 : 0;
   P.nk = K / SKc;
   P.scale = scale;
   P.out = out;
   P.status = reinterpret_cast<uint32_t*>(ws);
+  CUtensorMap mA, mB;
+  constexpr auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!sh_map(&mA, x, uint64_t(G) * K, T, 1, SMt, BF) || !sh_map(&mB, qw, K, uint64_t(G) * N, 1, P.bn, BF))
+    return cudaErrorInvalidValue;
+  set_smem(k_sh_gemm, kSSmem);
   return launch_kernel("lin_gemm", k_sh_gemm, dim3(std::min(sms, P.ntiles)), dim3(kSThreads), kSSmem, st, true, P,
                        mA, mB);
 }

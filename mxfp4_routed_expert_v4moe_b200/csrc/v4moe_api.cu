@@ -251,23 +251,33 @@ int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const voi
                        stream);
 }
 
+size_t v4moe_linear_w8a16_grouped_workspace_bytes(int32_t T, int32_t G, int32_t N, int32_t K) {
+  if (T < 0 || G <= 0 || N <= 0 || K <= 0) return 0;
+  return linear_w8a16_ws_bytes(G, N, K);
+}
+
+int32_t v4moe_linear_w8a16_grouped(int32_t T, int32_t G, int32_t N, int32_t K, const void* x, const int8_t* q,
+                                   const float* scale, void* out, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || G <= 0 || N <= 0 || K <= 0 || N % 32 != 0 || K % 64 != 0) return V4MOE_ERR_INVALID_ARG;
+  if (int64_t(G) * N > (int64_t(1) << 30) || int64_t(G) * K > (int64_t(1) << 30)) return V4MOE_ERR_INVALID_ARG;
+  if (!q || !scale || !aligned(q, 16) || !aligned(scale, 4)) return V4MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !out || !aligned(x, 16) || !aligned(out, 16) || x == out)) return V4MOE_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256)) return V4MOE_ERR_INVALID_ARG;
+  if (ws_bytes < linear_w8a16_ws_bytes(G, N, K)) return V4MOE_ERR_WORKSPACE;
+  if (int32_t r = check_device()) return r;
+  if (T == 0) return V4MOE_OK;
+  return launch_status(launch_linear_w8a16(T, G, N, K, static_cast<const __nv_bfloat16*>(x), q, scale,
+                                           static_cast<__nv_bfloat16*>(out), static_cast<char*>(ws),
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 size_t v4moe_linear_w8a16_workspace_bytes(int32_t T, int32_t N, int32_t K) {
-  if (T < 0 || N <= 0 || K <= 0) return 0;
-  return linear_w8a16_ws_bytes(N, K);
+  return v4moe_linear_w8a16_grouped_workspace_bytes(T, 1, N, K);
 }
 
 int32_t v4moe_linear_w8a16(int32_t T, int32_t N, int32_t K, const void* x, const int8_t* q, const float* scale,
                            void* out, void* ws, size_t ws_bytes, void* stream) {
-  if (T < 0 || N <= 0 || K <= 0 || N % 32 != 0 || K % 64 != 0) return V4MOE_ERR_INVALID_ARG;
-  if (!q || !scale || !aligned(q, 16) || !aligned(scale, 4)) return V4MOE_ERR_INVALID_ARG;
-  if (T > 0 && (!x || !out || !aligned(x, 16) || !aligned(out, 16) || x == out)) return V4MOE_ERR_INVALID_ARG;
-  if (!ws || !aligned(ws, 256)) return V4MOE_ERR_INVALID_ARG;
-  if (ws_bytes < linear_w8a16_ws_bytes(N, K)) return V4MOE_ERR_WORKSPACE;
-  if (int32_t r = check_device()) return r;
-  if (T == 0) return V4MOE_OK;
-  return launch_status(launch_linear_w8a16(T, N, K, static_cast<const __nv_bfloat16*>(x), q, scale,
-                                           static_cast<__nv_bfloat16*>(out), static_cast<char*>(ws),
-                                           static_cast<cudaStream_t>(stream)));
+  return v4moe_linear_w8a16_grouped(T, 1, N, K, x, q, scale, out, ws, ws_bytes, stream);
 }
 
 int32_t v4moe_read_device_status(const void* ws, void* stream) {

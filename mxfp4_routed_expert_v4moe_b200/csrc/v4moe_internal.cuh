@@ -161,11 +161,12 @@ bool sh_supported(const v4moe_config& c, int64_t T);
 cudaError_t launch_sh_w13(const ForwardArgs& a, const __half* x16, const int* sigma, char* sh16, cudaStream_t st);
 cudaError_t launch_sh_w2_combine(const ForwardArgs& a, char* sh16, cudaStream_t st);
 
-// W8A16 linear: out[t, n] = bf16(scale[n] * sum_k q[n, k] x[t, k]); the int8
-// weights are widened to bf16 in ws (after its 256-byte status block).
-size_t linear_w8a16_ws_bytes(int64_t N, int64_t K);
-cudaError_t launch_linear_w8a16(int T, int N, int K, const __nv_bfloat16* x, const int8_t* q, const float* scale,
-                                __nv_bfloat16* out, char* ws, cudaStream_t st);
+// W8A16 linear in G groups: out[t, g N + n] = bf16(scale[g N + n] *
+// sum_k q[g N + n, k] x[t, g K + k]); the int8 weights are widened to bf16 in
+// ws (after its 256-byte status block).
+size_t linear_w8a16_ws_bytes(int64_t G, int64_t N, int64_t K);
+cudaError_t launch_linear_w8a16(int T, int G, int N, int K, const __nv_bfloat16* x, const int8_t* q,
+                                const float* scale, __nv_bfloat16* out, char* ws, cudaStream_t st);
 
 // Tensor-core path (tcgen05 grouped GEMMs) for larger token counts.
 cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, char* sh16,

@@ -222,3 +222,18 @@ def linear_w8a16(x_bf16: np.ndarray, q: np.ndarray, scale: np.ndarray, rows=None
     out = np.zeros((T, N), np.float64)
     lib().orc_linear_w8a16(T, N, K, _p(x), _p(q), _p(scale), _p(out))
     return out
+
+
+def linear_w8a16_grouped(x_bf16: np.ndarray, q: np.ndarray, scale: np.ndarray, G: int, rows=None) -> np.ndarray:
+    """The W8A16 linear in G independent groups (the config's wo_a: o_groups
+    groups of heads, each with its own block of rows of one int8 matrix):
+    out[t, g N + n] = sum_k x[t, g K + k] q[g N + n, k] scale[g N + n].
+    x_bf16: [T, G K]; q: [G N, K]; scale: [G N]. Each group is the plain linear
+    on its slice of columns and rows."""
+    T, GK = x_bf16.shape
+    GN, K = q.shape
+    assert GK == G * K and GN % G == 0
+    N = GN // G
+    parts = [linear_w8a16(x_bf16[:, g * K:(g + 1) * K], q[g * N:(g + 1) * N], scale[g * N:(g + 1) * N], rows=rows)
+             for g in range(G)]
+    return np.concatenate(parts, axis=1)

@@ -90,4 +90,9 @@ def test_linear_w8a16_rejects_bad_shapes_before_any_launch():
     assert V.v4moe_linear_w8a16(4, 64, 96, 16, 16, 16, 32, 256, 1 << 20, 0) == V.V4MOE_ERR_INVALID_ARG
     assert V.v4moe_linear_w8a16(4, 64, 128, 16, 8, 16, 32, 256, 1 << 20, 0) == V.V4MOE_ERR_INVALID_ARG
     assert V.v4moe_linear_w8a16(4, 64, 128, 16, 16, 16, 32, 256, 100, 0) == V.V4MOE_ERR_WORKSPACE
+    assert V.v4moe_linear_w8a16_grouped_workspace_bytes(4, 8, 64, 128) == 256 + 8 * 64 * 128 * 2
+    assert V.v4moe_linear_w8a16_grouped_workspace_bytes(4, 0, 64, 128) == 0
+    assert V.v4moe_linear_w8a16_grouped(4, 0, 64, 128, 16, 16, 16, 32, 256, 1 << 20, 0) == V.V4MOE_ERR_INVALID_ARG
+    assert V.v4moe_linear_w8a16_grouped(4, 2, 48, 128, 16, 16, 16, 32, 256, 1 << 20, 0) == V.V4MOE_ERR_INVALID_ARG
+    assert V.v4moe_linear_w8a16_grouped(4, 2, 64, 128, 16, 16, 16, 32, 256, 1000, 0) == V.V4MOE_ERR_WORKSPACE
 

@@ -17,22 +17,30 @@ pytestmark = pytest.mark.gpu
 torch = pytest.importorskip("torch")
 
 
-def _run(T, N, K, seed, rows=None):
+def _run(T, N, K, seed, rows=None, G=1):
     import mxfp4_routed_expert_v4moe_b200 as V
-    x_bits = IN.normal_bf16(seed, 1, T * K).reshape(T, K)
-    q, s = IN.int8_normal(seed, 2, N, K, 0.02)
+    x_bits = IN.normal_bf16(seed, 1, T * G * K).reshape(T, G * K)
+    q, s = IN.int8_normal(seed, 2, G * N, K, 0.02)
     x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)
     qd = torch.from_numpy(q).cuda()
     sd = torch.from_numpy(s).cuda()
-    out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-    nbytes = V.v4moe_linear_w8a16_workspace_bytes(T, N, K)
-    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
-    rc = V.v4moe_linear_w8a16(T, N, K, x, qd, sd, out, ws, nbytes)
+    out = torch.full((T, G * N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    if G == 1:
+        nbytes = V.v4moe_linear_w8a16_workspace_bytes(T, N, K)
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+        rc = V.v4moe_linear_w8a16(T, N, K, x, qd, sd, out, ws, nbytes)
+    else:
+        nbytes = V.v4moe_linear_w8a16_grouped_workspace_bytes(T, G, N, K)
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+        rc = V.v4moe_linear_w8a16_grouped(T, G, N, K, x, qd, sd, out, ws, nbytes)
     assert rc == V.V4MOE_OK, V.status_string(rc)
     assert V.v4moe_read_device_status(ws) == V.V4MOE_OK
     got = bf16_to_f64(out)
     rows = np.arange(T) if rows is None else np.asarray(rows)
-    ref = O.linear_w8a16(x_bits, q, s, rows=rows)
+    if G == 1:
+        ref = O.linear_w8a16(x_bits, q, s, rows=rows)
+    else:
+        ref = O.linear_w8a16_grouped(x_bits, q, s, G, rows=rows)
     assert np.isfinite(got).all()
     return got[rows], ref
 
@@ -50,6 +58,30 @@ def test_linear_attention_projection_shapes(name, N, K):
     rows = [0, 1, 128, 129, 255, 256]  # both token tiles and the ragged tail
     got, ref = _run(T, N, K, seed=11, rows=rows)
     assert_close(got, ref, name)
+
+
+def test_linear_tokens_outnumber_channels():
+    # more tokens than channels (token tiles walked inside a weight block's
+    # row of tiles) and exactly one wave of 256-row tiles with a ragged tail
+    T, N, K = 4700, 1024, 192
+    rows = [0, 127, 128, 2047, 4607, 4608, 4699]
+    got, ref = _run(T, N, K, seed=13, rows=rows)
+    assert_close(got, ref, "tokens > channels")
+
+
+@pytest.mark.parametrize("T,G,N,K", [(70, 3, 96, 128), (129, 2, 288, 192)])
+def test_linear_grouped_small(T, G, N, K):
+    got, ref = _run(T, N, K, seed=17, G=G)
+    assert_close(got, ref, f"grouped T={T} G={G} N={N} K={K}")
+
+
+def test_linear_grouped_wo_a_shape():
+    # wo_a: o_groups = 8 groups, o_lora_rank = 1024 outputs from the group's
+    # 8 heads x head_dim 512 = 4096 inputs
+    T = 257
+    rows = [0, 1, 128, 129, 255, 256]
+    got, ref = _run(T, 1024, 4096, seed=19, rows=rows, G=8)
+    assert_close(got, ref, "wo_a")
 
 
 def test_linear_empty_batch():

@@ -361,3 +361,24 @@ def test_linear_w8a16_matches_numpy_and_row_subset():
     got = O.linear_w8a16(x, q, s)
     assert np.allclose(got, ref, rtol=1e-13, atol=1e-15)
     assert np.array_equal(O.linear_w8a16(x, q, s, rows=[4, 1]), got[[4, 1]])
+
+
+def test_linear_w8a16_grouped_is_block_diagonal():
+    # G groups on their own column and row slices == one linear whose weight is
+    # block-diagonal (zeros between groups): checks which x columns and which
+    # weight rows each group takes
+    rng = np.random.default_rng(5)
+    T, G, N, K = 3, 3, 4, 8
+    x = bf16(rng.standard_normal((T, G * K)))
+    q = rng.integers(-127, 128, size=(G * N, K)).astype(np.int8)
+    s = (rng.random(G * N) * 0.01 + 0.001).astype(np.float32)
+    bd = np.zeros((G * N, G * K), np.int8)
+    for g in range(G):
+        bd[g * N:(g + 1) * N, g * K:(g + 1) * K] = q[g * N:(g + 1) * N]
+    got = O.linear_w8a16_grouped(x, q, s, G)
+    assert got.shape == (T, G * N)
+    assert np.allclose(got, O.linear_w8a16(x, bd, s), rtol=1e-14, atol=0)
+    ref = np.concatenate([bf16_val(x)[:, g * K:(g + 1) * K] @ (q[g * N:(g + 1) * N].astype(np.float64)
+                          * s[g * N:(g + 1) * N, None].astype(np.float64)).T for g in range(G)], axis=1)
+    assert np.allclose(got, ref, rtol=1e-13, atol=1e-15)
+    assert np.array_equal(O.linear_w8a16_grouped(x, q, s, G, rows=[2]), got[[2]])
