@@ -20,16 +20,18 @@
 //  * k_dec_w13: one CTA per SM, two groups of eight warps. Work items are w13
 //    slabs (8 channels of a routed expert: 8 gate rows and the 8 matching up
 //    rows; or 4 + 4 int8 rows of the shared expert), numbered shared first,
-//    then routed expert by expert; CTA b takes items b, b + G, ... as its ring
-//    positions 0, 1, .... Before the routing is known the CTA asks L2 for its
-//    shared slabs and for its share of the shared w2 rows; after it, for all
-//    of its routed slabs and its share of the routed w2 rows, so the HBM
-//    stream runs ahead of the shared-memory ring. Warp i of a group owns the
-//    128-wide K blocks i, i + 8, ... of a slab, multiplies them by the
-//    activations with mma.sync m16n8k16 (f16 operands, fp32 accumulation, the
-//    tokens as the 8 columns) and posts its partial tile to shared memory; the
-//    last warp to post sums the partials in warp order, refills the stage and
-//    writes h as f16 (routed: w * h).
+//    then routed expert by expert; CTA b takes a contiguous share of each as
+//    its ring positions 0, 1, .... The shared slabs do not depend on the
+//    routing: their copies are issued at the start and group 1 multiplies
+//    them while group 0 selects from the router's scores and builds the
+//    routing tables; then both groups take alternate positions of the routed
+//    slabs, and once its last slab is on its way the CTA asks L2 for its
+//    share of the routed w2 rows. Warp i of a group owns the 128-wide K
+//    blocks i, i + 8, ... of a slab, multiplies them by the activations with
+//    mma.sync m16n8k16 (f16 operands, fp32 accumulation, the tokens as the 8
+//    columns) and posts its partial tile to shared memory; the last warp to
+//    post sums the partials in warp order, refills the stage and writes h as
+//    f16 (routed: w * h).
 //  * k_dec_w2: two groups of eight warps, warp i of a group owning K blocks
 //    i, i + 8. CTA b owns a run of 16-row output blocks and goes through the
 //    shared expert and every routed expert for each of them, the two groups
@@ -429,7 +431,7 @@ struct W13Smem {
   uint64_t full[kStages13];
   int redcnt[kStages13];
   int lastfill[kStages13];
-  int sigma[8];
+  int sigma[2][8];  // per consumer group
   uint32_t xmax[2][kGW][8];
   float sh_scale[2][kShRows];  // gate / up row scales of this CTA's shared slabs
   Tables tb;
@@ -530,10 +532,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
   W13Smem& S = *reinterpret_cast<W13Smem*>(smem);
   char* stages = smem + kHead13;
   float4* parts = reinterpret_cast<float4*>(stages + size_t(kStages13) * P.stage_bytes);
+  // router scores and bias, outside the ring (it takes the shared slabs
+  // before the routing is known)
+  float* ssc = reinterpret_cast<float*>(reinterpret_cast<char*>(parts) + kPart13);
+  float* sbias = ssc + size_t(P.T) * P.E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = P.T, H = P.H;
   const int G = int(gridDim.x), b = int(blockIdx.x);
   const int n_s = P.Is > 0 ? P.Is / 4 : 0;
+  const bool learned = P.layer_mode && !P.token_ids;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages13; ++s) {
@@ -544,26 +551,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
     S.tb.nh = 0;
     fence_mbar_init();
   }
-  __syncthreads();
   // The w2 kernel may launch now (its CTAs start as these leave their SMs).
   pdl_launch_dependents();
-  // Global memory outside the ring is read before the first copy or L2
-  // request is issued: on this GPU a global load waits behind the SM's
-  // transfers in flight. The shared slabs' row scales:
-  {
-    const Chunk c0 = w13_chunk(P, 0, b, G);  // the shared range does not depend on the routing
-    for (int i = threadIdx.x; i < 4 * (c0.s1 - c0.s0) && i < kShRows; i += blockDim.x) {
-      S.sh_scale[0][i] = __ldg(P.sh13_scale + 4 * c0.s0 + i);
-      S.sh_scale[1][i] = __ldg(P.sh13_scale + P.Is + 4 * c0.s0 + i);
-    }
-  }
-
+  // The shared range of this CTA does not depend on the routing: its first
+  // nsp slabs go into the ring before the routing is known.
+  const Chunk c0 = w13_chunk(P, 0, b, G);
+  const int nsp = min(c0.s1 - c0.s0, kStages13);
   const int q = warp / kGW, wi = warp % kGW;
   const int g = lane >> 2, t = lane & 3;
   const int nkbH = H / 128;
-  // ---- x slices of this warp's K blocks for token g, then f16 scaled by 2^sigma
+
+  // Global memory outside the ring is read before the first copy is issued:
+  // on this GPU a global load waits behind the SM's transfers in flight. The
+  // loads of the shared slabs' row scales and the bias (into registers,
+  // stored to shared memory after the copies are issued) and of x go out
+  // first.
+  // Group 1 (which takes the shared slabs first) loads the row scales, group
+  // 0 (which selects) the bias, so each group's own barriers order the stores
+  // before its reads.
+  constexpr int kGT = kGW * 32;  // threads per group
+  const int nsr = min(4 * (c0.s1 - c0.s0), kShRows);
+  const int gt = int(threadIdx.x) - q * kGT;  // thread within the group
+  float rsg = 0.f, rsu = 0.f, rb[4] = {0.f, 0.f, 0.f, 0.f};
+  if (q == 1 && gt < nsr) {
+    rsg = __ldg(P.sh13_scale + 4 * c0.s0 + gt);
+    rsu = __ldg(P.sh13_scale + P.Is + 4 * c0.s0 + gt);
+  }
+  if (q == 0 && learned) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (gt + j * kGT < P.E) rb[j] = __ldg(P.bias + gt + j * kGT);
+    for (int i = gt + 4 * kGT; i < P.E; i += kGT) sbias[i] = __ldg(P.bias + i);
+  }
+  // this warp's x slices (token g; in L2 after the router)
   uint32_t B[kNJ][16];
-  uint32_t mx = 0u;
 #pragma unroll
   for (int j = 0; j < kNJ; ++j) {
     const int kb = wi + 8 * j;
@@ -581,18 +602,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) B[j][i] = 0u;
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) mx = absmax_bf16x2(mx, B[j][i]);
   }
-  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  if (t == 0) S.xmax[q][wi][g] = mx;
-  named_bar_sync(2 + q, kGW * 32);
+  __syncthreads();
+  if (warp == 14)
+    for (int p = 0; p < nsp; ++p)
+      fill13(P, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, c0.s0 + p), p);
+  if (q == 1 && gt < nsr) {
+    S.sh_scale[0][gt] = rsg;
+    S.sh_scale[1][gt] = rsu;
+  }
+  if (q == 0 && learned) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (gt + j * kGT < P.E) sbias[gt + j * kGT] = rb[j];
+  }
+  // ---- f16 activations scaled by 2^sigma (each group keeps its own copy)
   {
+    uint32_t mx = 0u;
+#pragma unroll
+    for (int j = 0; j < kNJ; ++j)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mx = absmax_bf16x2(mx, B[j][i]);
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if (t == 0) S.xmax[q][wi][g] = mx;
+    named_bar_sync(2 + q, kGW * 32);
     uint32_t rmx = 0u;
     for (int w = 0; w < kGW; ++w) rmx = max(rmx, S.xmax[q][w][g]);
     const int sg = sigma_of(rmx);
-    if (warp == 0 && t == 0) S.sigma[g] = sg;
+    if (wi == 0 && t == 0) S.sigma[q][g] = sg;
     const float mul = __int_as_float((sg + 127) << 23);
 #pragma unroll
     for (int j = 0; j < kNJ; ++j)
@@ -601,58 +639,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
         const __half2 hv = __floats2half2_rn(bf16_lo(B[j][i]) * mul, bf16_hi(B[j][i]) * mul);
         B[j][i] = *reinterpret_cast<const uint32_t*>(&hv);
       }
+    named_bar_sync(2 + q, kGW * 32);  // the group's sigma is visible to the group
   }
 
-  // ---- routing: every CTA selects from the scores and builds the tables. The
-  // scores and the bias are staged in the (still empty) ring.
-  float* ssc = reinterpret_cast<float*>(stages);
-  float* sbias = ssc + size_t(T) * P.E;
-  if (P.layer_mode && !P.token_ids) {
-    // the bias is an input: staged before the wait
-    for (int i = threadIdx.x; i < P.E; i += blockDim.x) sbias[i] = __ldg(P.bias + i);
-    __syncthreads();
-    // Run the selection once on whatever the ring holds, results discarded:
-    // its code is then cached when the scores arrive.
-    if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
-    __syncthreads();
-    if (warp == 0) route_tables(S.rt, S.tb, P, S.rt.sel_ids, S.rt.sel_w, true);
-  }
-  // the scores (previous grid) are complete and visible past this point
-  pdl_wait();
-  if (P.layer_mode) {
-    for (int i = threadIdx.x; i < T * P.E; i += blockDim.x) ssc[i] = __ldcg(P.scores + i);
-    __syncthreads();
-    if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
-    __syncthreads();
-    if (warp == 0) route_tables(S.rt, S.tb, P, S.rt.sel_ids, S.rt.sel_w, true);
-  } else if (warp == 0) {
-    route_tables(S.rt, S.tb, P, P.topk_ids, P.topk_w, b != 0);
-  }
-  __syncthreads();
-  if (b == 0) {  // one CTA writes the routing outputs and the w2 kernel's tables
-    if (warp == 0) publish_tables(S.tb, P);
-    if (P.layer_mode && warp == 1)
-      for (int i = lane; i < T * P.k; i += 32) {
-        P.topk_ids[i] = S.rt.sel_ids[i];
-        P.topk_w[i] = S.rt.sel_w[i];
-      }
-    if (P.layer_mode && warp == 2) write_permutation(S.rt, P, S.tb.nh);
-  }
-  const Chunk ch = w13_chunk(P, S.tb.nh, b, G);
-  const int npos = ch.size();
-  // The routed slabs stream through the ring; the routed w2 rows of this CTA's
-  // share are asked for once its last slab is on its way.
-  if (warp == 14) {
-    for (int p = 0; p < kStages13 && p < npos; ++p)
-      fill13(P, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, ch.item(p, n_s)), p);
-    if (npos <= kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
-  }
-
-  // ---- item loop: group q takes ring positions q, q + 2, ...
-  for (int pos = q; pos < npos; pos += 2) {
+  // One slab at ring position pos (chunk ch of npos positions): the warp's K
+  // blocks, its partial tile posted to shared memory; the last warp of the
+  // group to post sums the partials in warp order, refills the stage with
+  // position pos + kStages13 when `refill`, and writes h. False after a
+  // timed-out wait.
+  auto run_item = [&](const Chunk& ch, int npos, int pos, bool refill) -> bool {
     const Item m = w13_item(P, S.tb, ch.item(pos, n_s));
     const int s = pos % kStages13;
-    if (!__all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / kStages13) & 1u, P))) break;
+    if (!__all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / kStages13) & 1u, P))) return false;
     const char* st = stages + size_t(s) * P.stage_bytes;
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
     float4 p0;
@@ -674,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
     int old = 0;
     if (lane == 0) old = atomicAdd(&S.redcnt[s], 1);
     old = __shfl_sync(0xffffffffu, old, 0);
-    if (old != kGW - 1) continue;
+    if (old != kGW - 1) return true;
     // Last of the group: the stage and its partials are this warp's alone.
     __threadfence_block();
     float4 d = part[lane];
@@ -688,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
     }
     if (lane == 0) S.redcnt[s] = 0;
     __syncwarp();
-    if (pos + kStages13 < npos) {
+    if (refill && pos + kStages13 < npos) {
       fill13(P, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, ch.item(pos + kStages13, n_s)),
              pos + kStages13);
       if (pos + kStages13 == npos - 1 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
@@ -700,7 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
       for (int qq = 0; qq < 2; ++qq) {
         const int tok = 2 * t + qq;
         if (tok < T && ((mask >> tok) & 1u)) {
-          const float inv = pow2f(-S.sigma[tok]);
+          const float inv = pow2f(-S.sigma[q][tok]);
           const float h = clamped_swiglu_f(dg[qq] * inv, du[qq] * inv, P.limit) * S.tb.w[m.li * 8 + tok];
           P.dh[(size_t(m.li) * T + tok) * P.I + m.row0 + g] = __float2half_rn(h);
         }
@@ -713,13 +711,59 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
       for (int qq = 0; qq < 2; ++qq) {
         const int tok = 2 * t + qq;
         if (tok < T) {
-          const float inv = pow2f(-S.sigma[tok]);
+          const float inv = pow2f(-S.sigma[q][tok]);
           P.hs[size_t(tok) * P.Is + m.row0 + g] =
               __float2half_rn(clamped_swiglu_f(dg[qq] * sg * inv, du[qq] * su * inv, P.limit));
         }
       }
     }
+    return true;
+  };
+
+  bool ok = true;
+  if (q == 1) {
+    // ---- group 1: the shared slabs already on their way, while group 0 routes
+    for (int pos = 0; pos < nsp && ok; ++pos) ok = run_item(c0, nsp, pos, false);
+  } else {
+    // ---- group 0: routing. Every CTA selects from the scores and builds the
+    // tables; the scores (previous grid) are complete and visible past the wait.
+    pdl_wait();
+    if (P.layer_mode) {
+      for (int i = threadIdx.x; i < T * P.E; i += kGW * 32) ssc[i] = __ldcg(P.scores + i);
+      named_bar_sync(4, kGW * 32);
+      if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
+      named_bar_sync(4, kGW * 32);
+      if (warp == 0) route_tables(S.rt, S.tb, P, S.rt.sel_ids, S.rt.sel_w, true);
+    } else if (warp == 0) {
+      route_tables(S.rt, S.tb, P, P.topk_ids, P.topk_w, b != 0);
+    }
+    named_bar_sync(4, kGW * 32);
+    if (b == 0) {  // one CTA writes the routing outputs and the w2 kernel's tables
+      if (warp == 0) publish_tables(S.tb, P);
+      if (P.layer_mode && warp == 1)
+        for (int i = lane; i < T * P.k; i += 32) {
+          P.topk_ids[i] = S.rt.sel_ids[i];
+          P.topk_w[i] = S.rt.sel_w[i];
+        }
+      if (P.layer_mode && warp == 2) write_permutation(S.rt, P, S.tb.nh);
+    }
   }
+  __syncthreads();  // the tables are visible to both groups; stages [0, nsp) are free
+
+  const Chunk ch = w13_chunk(P, S.tb.nh, b, G);
+  const int npos = ch.size();
+  // Positions [nsp, nsp + kStages13) into the free stages; the routed w2 rows
+  // of this CTA's share are asked for once its last slab is on its way.
+  if (warp == 14 && ok) {
+    for (int p = nsp; p < nsp + kStages13 && p < npos; ++p)
+      fill13(P, S, stages + size_t(p % kStages13) * P.stage_bytes, p % kStages13,
+             w13_item(P, S.tb, ch.item(p, n_s)), p);
+    if (npos <= nsp + kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
+  }
+  ok = __syncthreads_and(ok);
+
+  // ---- item loop: group q takes ring positions nsp + q, nsp + q + 2, ...
+  for (int pos = nsp + q; pos < npos && ok; pos += 2) ok = run_item(ch, npos, pos, true);
   // No copy may still be landing in this CTA's shared memory (possible only
   // after a timeout).
   __syncthreads();
@@ -966,15 +1010,15 @@ Plan make_plan(const v4moe_config& c, int T) {
   int s13 = 16 * (H / 2) + 16 * (H / 32);
   if (Is > 0) s13 = std::max(s13, 8 * H);
   p.stage13 = (s13 + 127) / 128 * 128;
-  p.smem13 = kHead13 + size_t(kStages13) * p.stage13 + kPart13;
+  const size_t route_stage = (size_t(T) * c.n_experts + c.n_experts) * 4;  // scores + bias
+  p.smem13 = kHead13 + size_t(kStages13) * p.stage13 + kPart13 + (route_stage + 127) / 128 * 128;
   const int hoff = std::max(16 * Is, 16 * (I / 2) + 16 * (I / 32));
   const int s2 = hoff + T * std::max(I, Is) * 2;
   p.stage2 = (s2 + 127) / 128 * 128;
   const size_t room = 227 * 1024 - kHead2 - kRed2;
   p.nst2 = int(std::min<size_t>(kMaxStages2, room / p.stage2));
   p.smem2 = kHead2 + size_t(p.nst2) * p.stage2 + kRed2;
-  const size_t route_stage = (size_t(T) * c.n_experts + c.n_experts) * 4;  // scores + bias in the ring
-  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 && route_stage <= size_t(kStages13) * p.stage13 &&
+  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 &&
          size_t(T) * H * 2 <= 227 * 1024;
   return p;
 }
