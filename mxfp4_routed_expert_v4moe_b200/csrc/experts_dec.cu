@@ -263,8 +263,8 @@ struct RouteSmem {
 // The batch's routed experts in ascending id, per (expert, token) weights and
 // token masks, from topk ids / weights (global or shared memory), into tb;
 // one warp. Out-of-range ids are skipped and, unless `quiet`, flagged.
-__device__ __noinline__ void route_tables(RouteSmem& S, Tables& tb, const DecParams& P, const int32_t* tids, const float* tw,
-                             bool quiet) {
+__device__ __forceinline__ void route_tables(RouteSmem& S, Tables& tb, const DecParams& P, const int32_t* tids,
+                                             const float* tw, bool quiet) {
   const int lane = threadIdx.x & 31;
   const int Sn = P.T * P.k;
   S.bits[lane] = 0u;
@@ -369,8 +369,10 @@ __device__ __noinline__ void write_permutation(RouteSmem& S, const DecParams& P,
 }
 
 // Top-k selection of token t (one warp) from scores and bias in shared memory,
-// into the RouteSmem selection arrays.
-__device__ __noinline__ void select_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
+// into the RouteSmem selection arrays. Inlined: the routing runs while the
+// shared slabs' copies are in flight, and on this GPU the local-memory traffic
+// of a call (saved registers) would wait behind them.
+__device__ __forceinline__ void select_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
                                              const float* sbias) {
   if (P.token_ids)
     select_hash_warp<true>(t, P.E, P.k, P.vocab, P.routed_scale, ssc + size_t(t) * P.E, P.token_ids, P.tid2eid,
@@ -436,6 +438,7 @@ struct W13Smem {
   float sh_scale[2][kShRows];  // gate / up row scales of this CTA's shared slabs
   Tables tb;
   RouteSmem rt;
+  int ready;          // group 0 has built the tables
 };
 
 constexpr size_t kHead13 = (sizeof(W13Smem) + 127) / 128 * 128;
@@ -549,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
       S.lastfill[s] = -1;
     }
     S.tb.nh = 0;
+    S.ready = 0;
     fence_mbar_init();
   }
   // The w2 kernel may launch now (its CTAs start as these leave their SMs).
@@ -583,26 +587,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
       if (gt + j * kGT < P.E) rb[j] = __ldg(P.bias + gt + j * kGT);
     for (int i = gt + 4 * kGT; i < P.E; i += kGT) sbias[i] = __ldg(P.bias + i);
   }
-  // this warp's x slices (token g; in L2 after the router)
+  // this warp's x slices (token g; in L2 after the router), loaded by each
+  // group when it is about to use them: group 1 at once, group 0 after the
+  // routing, so that the routing code runs with few live registers and no
+  // local-memory traffic (on this GPU that would wait behind the copies in
+  // flight)
   uint32_t B[kNJ][16];
-#pragma unroll
-  for (int j = 0; j < kNJ; ++j) {
-    const int kb = wi + 8 * j;
-    if (kb < nkbH && g < T) {
-      const uint4* src = reinterpret_cast<const uint4*>(P.x + size_t(g) * H + kb * 128 + 32 * t);
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const uint4 v = __ldg(src + p);
-        B[j][4 * p] = v.x;
-        B[j][4 * p + 1] = v.y;
-        B[j][4 * p + 2] = v.z;
-        B[j][4 * p + 3] = v.w;
+  auto load_x = [&]() {
+  #pragma unroll
+    for (int j = 0; j < kNJ; ++j) {
+      const int kb = wi + 8 * j;
+      if (kb < nkbH && g < T) {
+        const uint4* src = reinterpret_cast<const uint4*>(P.x + size_t(g) * H + kb * 128 + 32 * t);
+  #pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const uint4 v = __ldg(src + p);
+          B[j][4 * p] = v.x;
+          B[j][4 * p + 1] = v.y;
+          B[j][4 * p + 2] = v.z;
+          B[j][4 * p + 3] = v.w;
+        }
+      } else {
+  #pragma unroll
+        for (int i = 0; i < 16; ++i) B[j][i] = 0u;
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) B[j][i] = 0u;
     }
-  }
+  };
   __syncthreads();
   if (warp == 14)
     for (int p = 0; p < nsp; ++p)
@@ -617,7 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
       if (gt + j * kGT < P.E) sbias[gt + j * kGT] = rb[j];
   }
   // ---- f16 activations scaled by 2^sigma (each group keeps its own copy)
-  {
+  auto prep_x = [&]() {
+    load_x();
     uint32_t mx = 0u;
 #pragma unroll
     for (int j = 0; j < kNJ; ++j)
@@ -640,14 +651,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
         B[j][i] = *reinterpret_cast<const uint32_t*>(&hv);
       }
     named_bar_sync(2 + q, kGW * 32);  // the group's sigma is visible to the group
-  }
+  };
 
   // One slab at ring position pos (chunk ch of npos positions): the warp's K
   // blocks, its partial tile posted to shared memory; the last warp of the
   // group to post sums the partials in warp order, refills the stage with
   // position pos + kStages13 when `refill`, and writes h. False after a
   // timed-out wait.
-  auto run_item = [&](const Chunk& ch, int npos, int pos, bool refill) -> bool {
+  auto run_item = [&](const Chunk& ch, int npos, int pos, bool refill, bool need_tables) -> bool {
     const Item m = w13_item(P, S.tb, ch.item(pos, n_s));
     const int s = pos % kStages13;
     if (!__all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / kStages13) & 1u, P))) return false;
@@ -686,10 +697,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
     }
     if (lane == 0) S.redcnt[s] = 0;
     __syncwarp();
-    if (refill && pos + kStages13 < npos) {
-      fill13(P, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, ch.item(pos + kStages13, n_s)),
-             pos + kStages13);
-      if (pos + kStages13 == npos - 1 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
+    if (refill) {
+      Chunk cr = ch;
+      int nr = npos;
+      bool have = true;
+      if (need_tables) {  // the next position may be routed: wait for the tables
+        uint32_t i = 0;
+        while (*reinterpret_cast<volatile int*>(&S.ready) == 0 && ++i < kBarTries) __nanosleep(32);
+        have = i < kBarTries;
+        if (!have && lane == 0) atomicOr(P.status, kStatusTimeout);
+        __threadfence_block();
+        cr = w13_chunk(P, S.tb.nh, b, G);
+        nr = cr.size();
+      }
+      if (have && pos + kStages13 < nr) {
+        fill13(P, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, cr.item(pos + kStages13, n_s)),
+               pos + kStages13);
+        if (pos + kStages13 == nr - 1 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
+      }
+      if (!have) return false;
     }
     const float dg[2] = {d.x, d.y}, du[2] = {d.z, d.w};
     if (m.kind == kR13) {
@@ -722,48 +748,61 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
 
   bool ok = true;
   if (q == 1) {
-    // ---- group 1: the shared slabs already on their way, while group 0 routes
-    for (int pos = 0; pos < nsp && ok; ++pos) ok = run_item(c0, nsp, pos, false);
+    // ---- group 1: the shared slabs already on their way, while group 0
+    // routes; their refills continue with the following positions
+    prep_x();
+    for (int pos = 0; pos < nsp && ok; ++pos) ok = run_item(c0, nsp, pos, true, true);
   } else {
     // ---- group 0: routing. Every CTA selects from the scores and builds the
     // tables; the scores (previous grid) are complete and visible past the wait.
     pdl_wait();
     if (P.layer_mode) {
-      for (int i = threadIdx.x; i < T * P.E; i += kGW * 32) ssc[i] = __ldcg(P.scores + i);
-      named_bar_sync(4, kGW * 32);
+      for (int i = threadIdx.x; i < T * P.E; i += kGT) ssc[i] = __ldcg(P.scores + i);
+      named_bar_sync(4, kGT);
       if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
-      named_bar_sync(4, kGW * 32);
+      named_bar_sync(4, kGT);
       if (warp == 0) route_tables(S.rt, S.tb, P, S.rt.sel_ids, S.rt.sel_w, true);
     } else if (warp == 0) {
       route_tables(S.rt, S.tb, P, P.topk_ids, P.topk_w, b != 0);
     }
-    named_bar_sync(4, kGW * 32);
+    named_bar_sync(4, kGT);
+    if (warp == 0) {
+      // the stages the shared slabs did not take, then the tables are ready
+      // for group 1's refills
+      const Chunk cr = w13_chunk(P, S.tb.nh, b, G);
+      const int nr = cr.size();
+      for (int p = nsp; p < kStages13 && p < nr; ++p)
+        fill13(P, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, cr.item(p, n_s)), p);
+      if (nr <= kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
+      __threadfence_block();
+      if (lane == 0) *reinterpret_cast<volatile int*>(&S.ready) = 1;
+    }
     if (b == 0) {  // one CTA writes the routing outputs and the w2 kernel's tables
-      if (warp == 0) publish_tables(S.tb, P);
-      if (P.layer_mode && warp == 1)
+      if (warp == 1) publish_tables(S.tb, P);
+      if (P.layer_mode && warp == 2)
         for (int i = lane; i < T * P.k; i += 32) {
           P.topk_ids[i] = S.rt.sel_ids[i];
           P.topk_w[i] = S.rt.sel_w[i];
         }
-      if (P.layer_mode && warp == 2) write_permutation(S.rt, P, S.tb.nh);
+      if (P.layer_mode && warp == 3) write_permutation(S.rt, P, S.tb.nh);
     }
+    prep_x();
   }
-  __syncthreads();  // the tables are visible to both groups; stages [0, nsp) are free
-
+  if (q == 1) {
+    // group 0's tables, before this group's first routed position
+    uint32_t i = 0;
+    while (*reinterpret_cast<volatile int*>(&S.ready) == 0 && ++i < kBarTries) __nanosleep(32);
+    if (i >= kBarTries) {
+      ok = false;
+      if (lane == 0) atomicOr(P.status, kStatusTimeout);
+    }
+    __threadfence_block();
+  }
   const Chunk ch = w13_chunk(P, S.tb.nh, b, G);
   const int npos = ch.size();
-  // Positions [nsp, nsp + kStages13) into the free stages; the routed w2 rows
-  // of this CTA's share are asked for once its last slab is on its way.
-  if (warp == 14 && ok) {
-    for (int p = nsp; p < nsp + kStages13 && p < npos; ++p)
-      fill13(P, S, stages + size_t(p % kStages13) * P.stage_bytes, p % kStages13,
-             w13_item(P, S.tb, ch.item(p, n_s)), p);
-    if (npos <= nsp + kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
-  }
-  ok = __syncthreads_and(ok);
 
   // ---- item loop: group q takes ring positions nsp + q, nsp + q + 2, ...
-  for (int pos = nsp + q; pos < npos && ok; pos += 2) ok = run_item(ch, npos, pos, true);
+  for (int pos = nsp + q; pos < npos && ok; pos += 2) ok = run_item(ch, npos, pos, true, false);
   // No copy may still be landing in this CTA's shared memory (possible only
   // after a timeout).
   __syncthreads();
