@@ -142,23 +142,23 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
-def csrc_hash():
-    h = hashlib.sha256()
-    d = os.path.join(ROOT, "mxfp4_routed_expert_v4moe_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        h.update(open(os.path.join(d, f), "rb").read())
-    return h.hexdigest()[:16]
+def source_hash(fname):
+    """Hash of one kernel source file under csrc/ (the file the kernel lives in)."""
+    path = os.path.join(ROOT, "mxfp4_routed_expert_v4moe_b200", "csrc", fname)
+    if not os.path.exists(path):
+        return None
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
 
 def recorded_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu summary, if it matches this source."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's
+    source file is unchanged since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        d = json.load(open(p))
-        e = d.get(f"{kernel}@{workload}")
-        if e and e.get("csrc") == csrc_hash():
+        e = json.load(open(p)).get(f"{kernel}@{workload}")
+        if e and e.get("hash") == source_hash(e.get("file", "")):
             return e.get("bytes_per_launch")
     except Exception:
         return None
@@ -385,7 +385,8 @@ def run_linear(args):
                        "l2": "flushed between timed steps (512 MiB write, then 256 MiB read)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
                          "frac": achieved / pk["bf16"], "peak_src": pk["src"], "kernel": "lin_gemm",
-                         "kernel_ms": gemm_ms, "algorithmic_per_launch": flops, "traffic": None},
+                         "kernel_ms": gemm_ms, "algorithmic_per_launch": flops,
+                         "traffic": recorded_traffic("lin_gemm", args.workload)},
             "layer_roofline": {"algorithmic_flops": flops, "algorithmic_bytes": lin_bytes,
                                "roofline_ms": max(flops / (pk["bf16"] * 1e12), lin_bytes / (pk["hbm"] * 1e9)) * 1e3},
             "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches_per_step": v[1] / args.steps}
