@@ -224,6 +224,46 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_env():
+    """(world, rank, local_rank) from the launcher's environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_ranks(world, dev, backend="nccl"):
+    """One process per GPU: the process group (short timeout) when world > 1."""
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        kw = {"device_id": dev} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(values, world, dev):
+    """Element-wise maximum over ranks of a list of floats (device times)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def close_ranks(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def oracle_sample(wl, li, n_tok, seconds):
     """Time the oracle (route + layer) on n_tok tokens of the workload, repeated
     until about `seconds` of CPU time; returns (tokens/s, tokens, reps, secs)."""
@@ -306,17 +346,16 @@ def run_reference(args):
 
 
 def run_linear(args):
-    """One W8A16 linear call per step (v4moe_linear_w8a16), same timing rules."""
+    """One W8A16 linear call per step (v4moe_linear_w8a16_grouped), same timing rules."""
     import torch
 
     import inputs as IN
     import mxfp4_routed_expert_v4moe_b200 as V
     T, G, N, K = LINEAR_WORKLOADS[args.workload]
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    init_ranks(world, dev)
     x_bits = IN.normal_bf16(0, 1, T * G * K).reshape(T, G * K)
     q, sc = IN.int8_normal(0, 2, G * N, K, 0.02)
     x = torch.from_numpy(x_bits.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -341,6 +380,8 @@ def run_linear(args):
     clocks = ClockSampler(str(torch.cuda.get_device_properties(dev).uuid))
     clocks.start()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
     launches0 = V.v4moe_launch_count()
     for i in range(args.steps):
         flush_l2(i)
@@ -349,7 +390,8 @@ def run_linear(args):
         evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
     launches = V.v4moe_launch_count() - launches0
-    ms_step = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    barrier(world)
+    ms_total = sum(a.elapsed_time(b) for a, b in evs)
     x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     out_host = torch.empty((T, G * N), dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty_like(x)
@@ -362,8 +404,11 @@ def run_linear(args):
         out_host.copy_(out, non_blocking=True)
         e2e_evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs) / args.steps
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs)
     clk = clocks.stop()
+    ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, dev)
+    ms_step = ms_total / args.steps
+    e2e_ms /= args.steps
     V.v4moe_profile_reset()
     V.v4moe_profile_enable(True)
     for i in range(args.steps):
@@ -377,7 +422,7 @@ def run_linear(args):
     gemm_ms = prof.get("lin_gemm", (0.0, 1))[0] / max(prof.get("lin_gemm", (0.0, 1))[1], 1)
     achieved = flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
     lin_bytes = G * (N * K + 4 * N + 2 * T * K + 2 * T * N)
-    line = {"metric": LINEAR_METRIC, "value": T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world,
+    line = {"metric": LINEAR_METRIC, "value": T * world / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": args.workload, "T": T, "G": G, "N": N, "K": K,
@@ -391,7 +436,7 @@ def run_linear(args):
                                "roofline_ms": max(flops / (pk["bf16"] * 1e12), lin_bytes / (pk["hbm"] * 1e9)) * 1e3},
             "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches_per_step": v[1] / args.steps}
                         for k, v in sorted(prof.items(), key=lambda kv: -kv[1][0])},
-            "e2e": {"value": T / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(T * G * K * 2),
+            "e2e": {"value": T * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(T * G * K * 2),
                     "d2h_bytes_per_step": int(T * G * N * 2)},
             "gpu_launches": int(launches), "clocks": clk}
     line["layer_roofline"]["frac"] = line["layer_roofline"]["roofline_ms"] / ms_step
@@ -406,6 +451,7 @@ def run_linear(args):
                                 "sample": f"{reps} x {len(rows)} token rows of {args.workload}, {el:.1f} s single-threaded fp64"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    close_ranks(world)
 
 
 def main():
@@ -417,21 +463,15 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
     import torch
-    import torch.distributed as dist
 
     import inputs as IN
     import mxfp4_routed_expert_v4moe_b200 as V
     from mxfp4_routed_expert_v4moe_b200 import MoELayer
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
+    init_ranks(world, dev)
 
     wl = IN.WORKLOADS[args.workload]
     li = IN.make_layer_inputs(wl)
@@ -470,8 +510,7 @@ def main():
     # ---- timed region: K steps, L2 flushed between steps ----------------------
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     torch.cuda.synchronize(dev)
     launches0 = V.v4moe_launch_count()
     for i in range(args.steps):
@@ -481,8 +520,7 @@ def main():
         evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
     launches = V.v4moe_launch_count() - launches0
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     ms_total = sum(a.elapsed_time(b) for a, b in evs)
 
     # ---- end to end through the public API: pinned host in, host out ----------
@@ -516,10 +554,7 @@ def main():
     prof = V.v4moe_profile_read()
     V.v4moe_profile_enable(False)
 
-    t_ms = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_ms, op=dist.ReduceOp.MAX)
-    ms_total, e2e_ms = float(t_ms[0]), float(t_ms[1])
+    ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, dev)
     ms_step = ms_total / args.steps
     tokens_total = wl.T * world
     value = tokens_total / (ms_step / 1e3)
@@ -577,8 +612,7 @@ def main():
                                           f"{wl.E} experts + layer), {el:.1f} s single-threaded fp64"}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    close_ranks(world)
 
 
 if __name__ == "__main__":
