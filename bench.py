@@ -222,8 +222,6 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
-# ----------------------------------------------------------------------------- CPU oracle
-
 # ----------------------------------------------------------------------------- ranks
 
 def rank_env():
@@ -263,6 +261,8 @@ def close_ranks(world):
         import torch.distributed as dist
         dist.destroy_process_group()
 
+
+# ----------------------------------------------------------------------------- CPU oracle
 
 def oracle_sample(wl, li, n_tok, seconds):
     """Time the oracle (route + layer) on n_tok tokens of the workload, repeated
