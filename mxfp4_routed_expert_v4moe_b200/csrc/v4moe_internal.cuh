@@ -125,7 +125,6 @@ struct ForwardArgs {
   float* ys;
 };
 
-cudaError_t launch_forward_simt(const ForwardArgs& a, cudaStream_t st);
 cudaError_t launch_combine(const ForwardArgs& a, cudaStream_t st);
 // Routed experts on block-scaled tcgen05 MMA (MXFP4 weights as stored, the
 // activations as two E4M3 planes with E8M0 scales).
