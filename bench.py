@@ -52,6 +52,7 @@ LINEAR_WORKLOADS = {
     "linear_indexer_wq_b_4096": (4096, 1, 64 * 128, 1024),
     "linear_indexer_wkv_4096": (4096, 1, 128, 4096),
 }
+HEADLINE = "decode_b1"   # the full-size layer at decode batch 1
 L2_FLUSH_BYTES = 512 << 20
 L2_CLEAN_BYTES = 256 << 20
 
@@ -62,10 +63,14 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode_b1")
+    ap.add_argument("--workload", default=None,
+                    help="one workload only (default: the headline decode_b1 line with every "
+                         "workload of the layer in its 'workloads' block)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--check-ranks", action="store_true",
+                    help="start the ranks and check their plumbing on the CPU (gloo); measures nothing")
     return ap.parse_args()
 
 
@@ -264,12 +269,15 @@ def close_ranks(world):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def oracle_sample(wl, li, n_tok, seconds):
+def oracle_sample(wl, li, n_tok, seconds, threads=1):
     """Time the oracle (route + layer) on n_tok tokens of the workload, repeated
-    until about `seconds` of CPU time; returns (tokens/s, tokens, reps, secs)."""
+    until about `seconds` of wall time; the layer part splits the tokens over
+    `threads` host threads (each runs the single-threaded oracle on its share).
+    Returns (tokens/s, tokens, reps, secs). When n_tok exceeds the batch, the
+    batch's tokens are taken again (independent copies of the same work)."""
     import inputs as IN
     import oracle as O
-    toks = np.arange(min(n_tok, wl.T), dtype=np.int32)
+    toks = np.arange(n_tok, dtype=np.int32) % wl.T
     sub = IN.LayerInputs(wl=wl.with_T(len(toks)), x=np.ascontiguousarray(li.x[toks]), gate=li.gate,
                          bias=li.bias,
                          token_ids=None if li.token_ids is None else np.ascontiguousarray(li.token_ids[toks]),
@@ -280,12 +288,32 @@ def oracle_sample(wl, li, n_tok, seconds):
     reps, t0 = 0, time.perf_counter()
     while True:
         ids, w, _, _ = lay.route()
-        lay.moe_tokens(np.arange(len(toks)), ids, w, threads=1)
+        lay.moe_tokens(np.arange(len(toks)), ids, w, threads=threads)
         reps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
     return reps * len(toks) / el, len(toks), reps, el
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, li, seconds):
+    """The oracle on all host cores (one token per thread, the batch's tokens
+    taken again when it has fewer), with the single-core figure beside it."""
+    C = host_cores()
+    tps, ntk, reps, el = oracle_sample(wl, li, C, seconds, threads=C)
+    tps1, ntk1, reps1, el1 = oracle_sample(wl, li, 1, seconds / 2, threads=1)
+    return {"value": tps, "unit": "tokens/s", "cores": C, "kind": "oracle",
+            "sample": f"{reps} x {ntk} token(s) of {wl.name} (route over all {wl.E} experts + layer) "
+                      f"on {C} host threads, {el:.1f} s, fp64",
+            "single_core": {"value": tps1, "unit": "tokens/s", "cores": 1,
+                            "sample": f"{reps1} x {ntk1} token(s), {el1:.1f} s"}}
 
 
 # ----------------------------------------------------------------------------- main
@@ -317,29 +345,32 @@ def run_reference_linear(args):
 
 
 def run_reference(args):
+    """The oracle as it stands on the host cores (one token of the workload per
+    thread per step), same metric and workload as the GPU arm; rank 0 only."""
     import inputs as IN
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = IN.WORKLOADS[args.workload]
+    wl = IN.WORKLOADS[args.workload or HEADLINE]
     li = IN.make_layer_inputs(wl)
+    C = host_cores()
     step_times = []
-    n_tok = 1
     for i in range(args.warmup + args.steps):
-        tps, ntk, reps, el = oracle_sample(wl, li, n_tok, 0.0)
+        tps, ntk, reps, el = oracle_sample(wl, li, C, 0.0, threads=C)
         if i >= args.warmup:
             step_times.append(el / reps)
     ms = 1e3 * float(np.mean(step_times))
-    value = n_tok / (ms / 1e3)
+    value = C / (ms / 1e3)
+    import oracle as O
+    cfg = workload_config(wl, 1)
+    cfg["experts_hit"] = int(len(np.unique(O.Layer(li).route()[0]))) if wl.T <= 64 else wl.E
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
-                       "shared_inter": wl.Is, "routing": wl.routing},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{n_tok} token(s) of {wl.name} per step (route over all "
-                                       f"{wl.E} experts + {wl.k} routed experts + shared expert)"},
+            "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": C, "kind": "oracle",
+                             "sample": f"{C} token(s) of {wl.name} per step, one per host thread (route "
+                                       f"over all {wl.E} experts + {wl.k} routed experts + shared expert)"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -454,8 +485,191 @@ def run_linear(args):
     close_ranks(world)
 
 
+def workload_config(wl, world):
+    return {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
+            "shared_inter": wl.Is, "routing": wl.routing, "global_batch": wl.T * world,
+            "parallelism": f"replicas{world}",
+            "l2": "flushed between timed steps (512 MiB write, then 256 MiB read)",
+            "weights": "MXFP4 routed (E2M1 + E8M0/32), int8 shared, bf16 gate"}
+
+
+class Bench:
+    """Device state shared by the workloads: the L2 flush buffers, the stream,
+    one layer object per weight set (the full-size workloads share theirs)."""
+
+    def __init__(self, dev, world, args):
+        import torch
+        self.torch, self.dev, self.world, self.args = torch, dev, world, args
+        self.stream = torch.cuda.current_stream(dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.clean = torch.ones(L2_CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
+        self.layers = {}
+        self.weights = {}
+
+    def flush_l2(self, i):
+        # Write a buffer larger than L2, then read another one: the timed step
+        # starts with no useful data in L2 and no dirty lines left to write back.
+        self.flush.fill_(i & 0xFF)
+        self.clean.sum()
+
+    def inputs(self, wl):
+        import inputs as IN
+        from mxfp4_routed_expert_v4moe_b200 import MoELayer
+        key = (wl.H, wl.I, wl.E, wl.k, wl.Is, wl.w_std, wl.gate_std, wl.seed)
+        if key not in self.weights:
+            self.weights[key] = IN.make_weights(wl)
+        li = IN.make_layer_inputs(wl, weights=self.weights[key])
+        if key not in self.layers:
+            self.layers[key] = MoELayer.from_host(li, device=self.dev)
+        return li, self.layers[key]
+
+    def measure(self, wl, li, layer):
+        """Timed steps (inputs resident), the end-to-end pass (pinned host x in,
+        out back) and the per-kernel pass of one workload -> result dict."""
+        import mxfp4_routed_expert_v4moe_b200 as V
+        torch, dev, args, stream = self.torch, self.dev, self.args, self.stream
+        x = torch.from_numpy(li.x).view(torch.bfloat16).to(dev)
+        bias = None if li.bias is None else torch.from_numpy(li.bias).to(dev)
+        tok = None if li.token_ids is None else torch.from_numpy(li.token_ids).to(dev)
+        tab = None if li.tid2eid is None else torch.from_numpy(li.tid2eid).to(dev)
+
+        def step():
+            return layer(x, bias, tok, tab)
+
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        acc = algorithmic(wl, layer.buffers(wl.T)["topk_ids"].cpu().numpy(), li.token_ids)
+
+        # ---- timed region: K steps, L2 flushed between steps ----------------
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(self.world)
+        torch.cuda.synchronize(dev)
+        launches0 = V.v4moe_launch_count()
+        for i in range(args.steps):
+            self.flush_l2(i)
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        launches = V.v4moe_launch_count() - launches0
+        barrier(self.world)
+        ms_total = sum(a.elapsed_time(b) for a, b in evs)
+
+        # ---- end to end through the public API: pinned host in, host out ----
+        x_host = torch.from_numpy(li.x).view(torch.bfloat16).pin_memory()
+        tok_host = None if li.token_ids is None else torch.from_numpy(li.token_ids).pin_memory()
+        out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(x)
+        tok_dev = None if tok is None else torch.empty_like(tok)
+        e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+        for i in range(args.steps):
+            self.flush_l2(i)
+            e2e_evs[i][0].record(stream)
+            x_dev.copy_(x_host, non_blocking=True)
+            if tok_dev is not None:
+                tok_dev.copy_(tok_host, non_blocking=True)
+            out = layer(x_dev, bias, tok_dev, tab)
+            out_host.copy_(out, non_blocking=True)
+            e2e_evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs)
+
+        # ---- per-kernel timing pass (events around every kernel) ------------
+        V.v4moe_profile_reset()
+        V.v4moe_profile_enable(True)
+        for i in range(args.steps):
+            self.flush_l2(i)
+            step()
+        torch.cuda.synchronize(dev)
+        prof = V.v4moe_profile_read()
+        V.v4moe_profile_enable(False)
+
+        ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], self.world, dev)
+        ms_step = ms_total / args.steps
+        tokens_total = wl.T * self.world
+        pk = peaks()
+        decode = wl.T <= 64
+        # dominant kernel = most device time in the profiled pass
+        dom_name, (dom_ms, dom_n) = max(prof.items(), key=lambda kv: kv[1][0]) if prof else ("none", (0.0, 1))
+        kind = kernel_kind(dom_name)
+        per_launch_s = dom_ms / max(dom_n, 1) / 1e3
+        steps_per_launch = max(dom_n, 1) / args.steps
+        if decode or kind is None:
+            alg = acc["kernel_bytes"].get(kind, acc["step_bytes"]) / steps_per_launch
+            achieved = alg / per_launch_s / 1e9 if per_launch_s > 0 else 0.0
+            roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                    "frac": achieved / pk["hbm"], "peak_src": pk["src"]}
+        else:
+            alg = acc["kernel_flops"][kind] / steps_per_launch
+            achieved = alg / per_launch_s / 1e12 if per_launch_s > 0 else 0.0
+            roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
+                    "frac": achieved / pk["bf16"], "peak_src": pk["src"]}
+        roof.update(kernel=dom_name, kernel_ms=dom_ms / max(dom_n, 1), algorithmic_per_launch=alg,
+                    traffic=recorded_traffic(dom_name, wl.name))
+        step_s = ms_step / 1e3
+        t_hbm = acc["step_bytes"] / (pk["hbm"] * 1e9)
+        t_tc = acc["step_flops"] / (pk["bf16"] * 1e12)
+        layer_roof_s = max(t_hbm, t_tc)
+        cfg = workload_config(wl, self.world)
+        cfg["experts_hit"] = acc["n_hit"]
+        return {"ms_per_step": ms_step, "value": tokens_total / step_s, "config": cfg,
+                "layer_roofline": {"algorithmic_bytes": acc["step_bytes"],
+                                   "algorithmic_flops": acc["step_flops"],
+                                   "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                                   "roofline_ms": layer_roof_s * 1e3,
+                                   "frac": layer_roof_s / step_s,
+                                   "achieved_GBps": acc["step_bytes"] / step_s / 1e9,
+                                   "achieved_TFLOPs": acc["step_flops"] / step_s / 1e12},
+                "roofline": roof,
+                "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches_per_step": v[1] / args.steps}
+                            for k, v in sorted(prof.items(), key=lambda kv: -kv[1][0])},
+                "e2e": {"value": tokens_total / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
+                        "h2d_bytes_per_step": int(x_host.numel() * 2 +
+                                                  (0 if tok_host is None else tok_host.numel() * 4)),
+                        "d2h_bytes_per_step": int(out_host.numel() * 2)},
+                "gpu_launches": int(launches)}
+
+
+def free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_command(n, argv):
+    """The torch.distributed.run command that starts n ranks of this script
+    (one process per GPU) with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(free_port()),
+            os.path.abspath(__file__), *argv]
+
+
+def check_ranks(args):
+    """The rank plumbing alone, on the CPU over gloo: every rank joins, the
+    per-rank numbers reduce to their maximum, rank 0 prints the count. No
+    measurement (nothing of the layer runs)."""
+    import torch
+    world, rank, _ = rank_env()
+    dev = torch.device("cpu")
+    init_ranks(world, dev, backend="gloo")
+    barrier(world)
+    got = max_over_ranks([float(rank + 1)], world, dev)
+    if rank == 0:
+        print(json.dumps({"check_ranks": True, "n_gpus": world, "ranks_joined": int(got[0])}), flush=True)
+    close_ranks(world)
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.impl == "ours":
+        # one process per GPU: start the ranks under torch.distributed.run
+        return subprocess.call(spawn_command(args.gpus, sys.argv[1:]))
+    if args.check_ranks:
+        return check_ranks(args)
     if args.workload in LINEAR_WORKLOADS:
         if args.impl == "reference":
             return run_reference_linear(args)
@@ -465,155 +679,55 @@ def main():
     import torch
 
     import inputs as IN
-    import mxfp4_routed_expert_v4moe_b200 as V
-    from mxfp4_routed_expert_v4moe_b200 import MoELayer
 
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     init_ranks(world, dev)
-
-    wl = IN.WORKLOADS[args.workload]
-    li = IN.make_layer_inputs(wl)
-    layer = MoELayer.from_host(li, device=dev)
-    x = torch.from_numpy(li.x).view(torch.bfloat16).to(dev)
-    bias = None if li.bias is None else torch.from_numpy(li.bias).to(dev)
-    tok = None if li.token_ids is None else torch.from_numpy(li.token_ids).to(dev)
-    tab = None if li.tid2eid is None else torch.from_numpy(li.tid2eid).to(dev)
-    stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    clean = torch.ones(L2_CLEAN_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def flush_l2(i):
-        # Write a buffer larger than L2, then read another one: the timed step
-        # starts with no useful data in L2 and no dirty lines left to write back.
-        flush.fill_(i & 0xFF)
-        clean.sum()
-
-    def step():
-        return layer(x, bias, tok, tab)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    ids_np = layer.buffers(wl.T)["topk_ids"].cpu().numpy()
-    acc = algorithmic(wl, ids_np, li.token_ids)
+    B = Bench(dev, world, args)
+    head_name = args.workload or HEADLINE
+    # the headline workload; with no --workload, every workload of the layer
+    # beside it (same weights for the full-size ones)
+    others = [] if args.workload else [w for w in IN.WORKLOAD_ORDER if w != head_name]
 
     uuid = None
     try:
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
+    wl = IN.WORKLOADS[head_name]
+    li, layer = B.inputs(wl)
     clocks = ClockSampler(uuid)
     clocks.start()
-
-    # ---- timed region: K steps, L2 flushed between steps ----------------------
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    launches0 = V.v4moe_launch_count()
-    for i in range(args.steps):
-        flush_l2(i)
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    launches = V.v4moe_launch_count() - launches0
-    barrier(world)
-    ms_total = sum(a.elapsed_time(b) for a, b in evs)
-
-    # ---- end to end through the public API: pinned host in, host out ----------
-    x_host = torch.from_numpy(li.x).view(torch.bfloat16).pin_memory()
-    tok_host = None if li.token_ids is None else torch.from_numpy(li.token_ids).pin_memory()
-    out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty_like(x)
-    tok_dev = None if tok is None else torch.empty_like(tok)
-    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush_l2(i)
-        e2e_evs[i][0].record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        if tok_dev is not None:
-            tok_dev.copy_(tok_host, non_blocking=True)
-        out = layer(x_dev, bias, tok_dev, tab)
-        out_host.copy_(out, non_blocking=True)
-        e2e_evs[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_evs)
+    r = B.measure(wl, li, layer)
     clk = clocks.stop()
 
-    # ---- per-kernel timing pass (events around every kernel) -----------------
-    V.v4moe_profile_reset()
-    V.v4moe_profile_enable(True)
-    for i in range(args.steps):
-        flush_l2(i)
-        step()
-    torch.cuda.synchronize(dev)
-    prof = V.v4moe_profile_read()
-    V.v4moe_profile_enable(False)
-
-    ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, dev)
-    ms_step = ms_total / args.steps
-    tokens_total = wl.T * world
-    value = tokens_total / (ms_step / 1e3)
-    e2e_value = tokens_total / (e2e_ms / args.steps / 1e3)
-
-    pk = peaks()
-    decode = wl.T <= 64
-    # dominant kernel = most device time in the profiled pass
-    dom_name, (dom_ms, dom_n) = max(prof.items(), key=lambda kv: kv[1][0]) if prof else ("none", (0.0, 1))
-    kind = kernel_kind(dom_name)
-    per_launch_s = dom_ms / max(dom_n, 1) / 1e3
-    steps_per_launch = max(dom_n, 1) / args.steps
-    if decode or kind is None:
-        alg = acc["kernel_bytes"].get(kind, acc["step_bytes"]) / steps_per_launch
-        achieved = alg / per_launch_s / 1e9 if per_launch_s > 0 else 0.0
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "peak_src": pk["src"]}
-    else:
-        alg = acc["kernel_flops"][kind] / steps_per_launch
-        achieved = alg / per_launch_s / 1e12 if per_launch_s > 0 else 0.0
-        roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16"], "peak_src": pk["src"]}
-    roof.update(kernel=dom_name, kernel_ms=dom_ms / max(dom_n, 1), algorithmic_per_launch=alg,
-                traffic=recorded_traffic(dom_name, wl.name))
-    step_s = ms_step / 1e3
-    layer_roof_s = max(acc["step_bytes"] / (pk["hbm"] * 1e9), acc["step_flops"] / (pk["bf16"] * 1e12))
-
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+    line = {"metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "I": wl.I, "E": wl.E, "k": wl.k,
-                       "shared_inter": wl.Is, "routing": wl.routing, "global_batch": wl.T * world,
-                       "parallelism": f"replicas{world}", "experts_hit": acc["n_hit"],
-                       "l2": "flushed between timed steps (512 MiB write, then 256 MiB read)",
-                       "weights": "MXFP4 routed (E2M1 + E8M0/32), int8 shared, bf16 gate"},
-            "layer_roofline": {"algorithmic_bytes": acc["step_bytes"],
-                               "algorithmic_flops": acc["step_flops"],
-                               "roofline_ms": layer_roof_s * 1e3,
-                               "frac": layer_roof_s / step_s,
-                               "achieved_GBps": acc["step_bytes"] / step_s / 1e9,
-                               "achieved_TFLOPs": acc["step_flops"] / step_s / 1e12},
-            "roofline": roof,
-            "kernels": {k: {"ms_per_launch": v[0] / max(v[1], 1), "launches_per_step": v[1] / args.steps}
-                        for k, v in sorted(prof.items(), key=lambda kv: -kv[1][0])},
-            "e2e": {"value": e2e_value, "unit": "tokens/s",
-                    "h2d_bytes_per_step": int(x_host.numel() * 2 + (0 if tok_host is None else tok_host.numel() * 4)),
-                    "d2h_bytes_per_step": int(out_host.numel() * 2)},
-            "gpu_launches": int(launches),
-            "clocks": clk}
+            "data": "synthetic", "config": r["config"], "layer_roofline": r["layer_roofline"],
+            "roofline": r["roofline"], "kernels": r["kernels"], "e2e": r["e2e"],
+            "gpu_launches": r["gpu_launches"], "clocks": clk}
+    if others:
+        block = {}
+        for name in others:
+            wlo = IN.WORKLOADS[name]
+            lio, layo = B.inputs(wlo)
+            ck = ClockSampler(uuid)
+            ck.start()
+            ro = B.measure(wlo, lio, layo)
+            ro["clocks"] = ck.stop()
+            block[name] = ro
+        block[head_name] = {k: r[k] for k in ("ms_per_step", "value", "config", "layer_roofline", "roofline",
+                                               "kernels", "e2e", "gpu_launches")}
+        block[head_name]["clocks"] = clk
+        line["workloads"] = {n: block[n] for n in IN.WORKLOAD_ORDER if n in block}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, ntk, reps, el = oracle_sample(wl, li, 1, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": f"{reps} x {ntk} token(s) of {wl.name} (route over all "
-                                          f"{wl.E} experts + layer), {el:.1f} s single-threaded fp64"}
+        line["cpu_baseline"] = cpu_baseline(wl, li, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     close_ranks(world)
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main() or 0)

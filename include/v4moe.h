@@ -147,8 +147,10 @@ int32_t v4moe_permute(const v4moe_config* cfg, int32_t T, const int32_t* topk_id
  *    V4MOE_ERR_INVALID_ARG before anything is launched.
  *  - It allocates nothing (no cudaMalloc/cudaFree, no allocating library
  *    call). The first call on a device looks up the array's device address
- *    with cudaGetSymbolAddress (once per device, with that device current);
- *    make that first call before any stream capture.
+ *    with cudaGetSymbolAddress (once per device, with that device current)
+ *    and keeps it for the life of the process; make that first call before
+ *    any stream capture. A device reset (cudaDeviceReset) after that first
+ *    call is not supported: the kept address would no longer be valid.
  *  - Every call shares the one array. Calls whose kernels may overlap on the
  *    GPU (different streams, or several host threads) race on it and must be
  *    serialised by the caller.
@@ -165,8 +167,12 @@ int32_t v4moe_permute_static(const v4moe_config* cfg, int32_t T, const int32_t* 
  * gate clamped above at swiglu_limit, up clamped on both sides). Routing may
  * come from v4moe_route/v4moe_permute or from the caller (offsets/sorted_slot/
  * slot_pos must be the permutation of topk_ids). x [T, H] bf16, out [T, H] bf16
- * (may not alias x). The intermediate h = swiglu(g, u) is rounded to bf16
- * before the down projection (W4A16: 16-bit activations). */
+ * (may not alias x). The intermediate h = swiglu(g, u) enters the down
+ * projection with at least 16-bit float precision (W4A16: 16-bit
+ * activations): as f16 on the decode and small-batch paths, and on the
+ * block-scaled tensor-core path as two E4M3 planes with E8M0 scales per 32
+ * channels, which hold an f16-rounded h exactly for values within 2^-14 of
+ * their block's largest magnitude (smaller ones keep their leading bits). */
 int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x,
                       const int32_t* topk_ids, const float* topk_w, const int32_t* offsets,
                       const int32_t* sorted_slot, const int32_t* slot_pos,

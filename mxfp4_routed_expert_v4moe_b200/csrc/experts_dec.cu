@@ -1079,9 +1079,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const v4moe_config& c = a.c;
   const Plan p = make_plan(c, a.T);
   if (!p.ok) return cudaErrorInvalidValue;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sms();
   DecParams P;
   P.T = a.T;
   P.H = c.hidden;

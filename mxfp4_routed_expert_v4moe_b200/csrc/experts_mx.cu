@@ -1078,9 +1078,7 @@ cudaError_t launch_mx_gemm(const ForwardArgs& a, int w2, const void* tiles, cons
     ok &= mx_map(&mBl, m.hq_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, c.inter, c.inter, S, 32);
   }
   if (!ok) return cudaErrorInvalidValue;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sms();
   // as many stages as fit next to the epilogue exchange and the barriers
   P.bn = bn;
   const int fixed = 2 * mx_scale_slot(bn) + kMXchBytes + kMBarBytes + kTileCacheBytes + 1024;
@@ -1139,9 +1137,7 @@ cudaError_t launch_mxt_gemm(const ForwardArgs& a, int w2, const void* tiles, con
     ok &= mx_map2d(&mSl, m.hs_lo, U8, I / 32, I / 32, S, 16, XM, NS);
   }
   if (!ok) return cudaErrorInvalidValue;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sms();
   set_smem(k_mxt_gemm, kXSmem);
   return launch_kernel(w2 ? "mxt_w2" : "mxt_w13", k_mxt_gemm, dim3(sms), dim3(kXThreads), kXSmem, st, true, P, mAh,
                        mAl, mB, mSw, mSh, mSl);

@@ -726,9 +726,7 @@ cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, cha
   (void)Isx;
   if (!ok) return cudaErrorInvalidValue;
 
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sms();
   set_smem(k_tc_gemm, kSmemBytes);
 
   TcParams P;

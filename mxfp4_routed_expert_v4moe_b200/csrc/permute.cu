@@ -232,20 +232,12 @@ extern "C" int32_t v4moe_permute_static(const v4moe_config* cfg, int32_t T, cons
                                         int32_t* counts, int32_t* offsets, int32_t* sorted_slot,
                                         int32_t* slot_pos, void* stream) {
   using namespace v4moe;
-  if (!cfg || T < 0 || cfg->top_k < 1 || cfg->top_k > 8 || cfg->n_experts < cfg->top_k ||
-      cfg->n_experts > 1024)
-    return V4MOE_ERR_INVALID_ARG;
+  // The same argument rules as v4moe_permute, plus the fixed array's limit.
+  if (!config_ok(cfg) || T < 0) return V4MOE_ERR_INVALID_ARG;
   if (!counts || !offsets) return V4MOE_ERR_INVALID_ARG;
   if (T > 0 && (!topk_ids || !sorted_slot || !slot_pos)) return V4MOE_ERR_INVALID_ARG;
   if (int64_t(T) * cfg->top_k > kStaticMaxSlots) return V4MOE_ERR_INVALID_ARG;
-  int dev = -1, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
-    cudaGetLastError();
-    return V4MOE_ERR_UNSUPPORTED_DEVICE;
-  }
-  if (major != 10 || minor != 0) return V4MOE_ERR_UNSUPPORTED_DEVICE;
+  if (int32_t r = check_device()) return r;
   cudaError_t err = cudaSuccess;
   int32_t* base = static_scratch(&err);
   if (!base) {

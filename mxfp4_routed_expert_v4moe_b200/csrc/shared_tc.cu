@@ -523,9 +523,7 @@ ShParams sh_params(const ForwardArgs& a, const int* sigma) {
 }
 
 int sm_count() {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sms();
   return sms;
 }
 

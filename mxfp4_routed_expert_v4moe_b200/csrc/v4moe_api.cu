@@ -8,10 +8,6 @@
 
 namespace v4moe {
 
-namespace {
-
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
 bool config_ok(const v4moe_config* c) {
   if (!c) return false;
   if (c->hidden <= 0 || c->hidden % 128 != 0) return false;
@@ -23,25 +19,53 @@ bool config_ok(const v4moe_config* c) {
   return true;
 }
 
-// Per-device compute capability cache.
-int32_t check_device() {
-  static std::mutex mu;
-  static std::unordered_map<int, bool> ok;
+namespace {
+struct DevInfo {
+  bool ok = false;
+  int sms = 0;
+};
+std::mutex g_dev_mu;
+std::unordered_map<int, DevInfo> g_dev;
+
+// The current device's cached attributes (queried once per device).
+const DevInfo* device_info() {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return V4MOE_ERR_UNSUPPORTED_DEVICE;
-  std::lock_guard<std::mutex> lock(mu);
-  auto it = ok.find(dev);
-  if (it == ok.end()) {
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
-      cudaGetLastError();
-      return V4MOE_ERR_UNSUPPORTED_DEVICE;
-    }
-    it = ok.emplace(dev, major == 10 && minor == 0).first;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return it->second ? V4MOE_OK : V4MOE_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  auto it = g_dev.find(dev);
+  if (it == g_dev.end()) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    DevInfo d;
+    d.ok = major == 10 && minor == 0;
+    d.sms = sms;
+    it = g_dev.emplace(dev, d).first;
+  }
+  return &it->second;
 }
+}  // namespace
+
+int32_t check_device() {
+  const DevInfo* d = device_info();
+  return d && d->ok ? V4MOE_OK : V4MOE_ERR_UNSUPPORTED_DEVICE;
+}
+
+int device_sms() {
+  const DevInfo* d = device_info();
+  return d && d->sms > 0 ? d->sms : 148;
+}
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int32_t check_ws(const v4moe_config* c, int32_t T, const void* ws, size_t ws_bytes) {
   if (!ws || !aligned(ws, 256)) return V4MOE_ERR_INVALID_ARG;

@@ -23,6 +23,13 @@ inline size_t align_up(size_t v, size_t a = kAlign) { return (v + a - 1) / a * a
 // Slots per chunk of the multi-CTA permutation.
 constexpr int kPermChunk = 2048;
 
+// Host checks shared by every entry point: the config's shape rules, and the
+// current device (compute capability 10.0). Device attributes are queried once
+// per device and cached (thread-safe); device_sms() is the cached SM count.
+bool config_ok(const v4moe_config* c);
+int32_t check_device();
+int device_sms();
+
 size_t tc_extra_bytes(const v4moe_config& c, int64_t T);
 
 // Router GEMM: the reduction is split so that about this many CTAs run; the

@@ -56,3 +56,23 @@ def test_single_rank_needs_no_process_group(monkeypatch):
     bench.barrier(w)
     assert bench.max_over_ranks([3.0, 4.0], w, torch.device("cpu")) == [3.0, 4.0]
     bench.close_ranks(w)
+
+
+def test_gpus_flag_starts_one_rank_per_gpu():
+    """`bench.py --gpus 2` with no launcher environment starts two ranks under
+    torch.distributed.run itself; both join and rank 0 reports n_gpus 2."""
+    import json
+    import subprocess
+    import sys
+
+    import bench
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    res = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--gpus", "2", "--check-ranks"],
+                         capture_output=True, text=True, timeout=300, env=env)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["ranks_joined"] == 2
+    cmd = bench.spawn_command(4, ["--steps", "3"])
+    assert "--nproc-per-node=4" in cmd and cmd[-2:] == ["--steps", "3"] and "127.0.0.1" in cmd

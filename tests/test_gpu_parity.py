@@ -7,8 +7,7 @@ import pytest
 
 import inputs as IN
 import oracle as O
-from parity_util import (NEAR_TIE, assert_close, bf16_to_f64, host_threads, sample_tokens,
-                         upload_activations)
+from parity_util import assert_close, bf16_to_f64, host_threads, run_parity, upload_activations
 
 pytestmark = pytest.mark.gpu
 
@@ -24,68 +23,6 @@ def _layer(li):
 def full_weights():
     """Full-size weights (identical for every full-size workload, seed 0)."""
     return IN.make_weights(IN.WORKLOADS["decode_b1"])
-
-
-def run_parity(li, layer, n_float_tokens=None, report=None):
-    wl = li.wl
-    T = wl.T
-    lay = O.Layer(li)
-    x, bias, tok, tab = upload_activations(li)
-    # --- routing -------------------------------------------------------------
-    ids_o, w_o, margin, _ = lay.route()
-    ids_g, w_g = layer.route(x, bias, tok, tab)
-    torch.cuda.synchronize()
-    ids_g = ids_g.cpu().numpy()
-    w_g = w_g.cpu().numpy().astype(np.float64)
-    near = margin < NEAR_TIE
-    ok = ~near
-    assert np.array_equal(ids_g[ok], ids_o[ok]), "router ids differ on non-tie tokens"
-    if ok.any():
-        assert_close(w_g[ok], w_o[ok], "topk_w")
-    # --- permutation on the oracle's ids (bit-exact) ---------------------------
-    ids_dev = torch.from_numpy(ids_o).cuda()
-    counts, offsets, sorted_slot, slot_pos = layer.permute(ids_dev)
-    c_o, off_o, ss_o, sp_o = O.permute(ids_o, wl.E)
-    torch.cuda.synchronize()
-    assert np.array_equal(counts.cpu().numpy(), c_o)
-    assert np.array_equal(offsets.cpu().numpy(), off_o)
-    S = T * wl.k
-    assert np.array_equal(sorted_slot.cpu().numpy()[:S], ss_o)
-    assert np.array_equal(slot_pos.cpu().numpy()[:S], sp_o)
-    # --- forward on the oracle's routing ---------------------------------------
-    w32 = w_o.astype(np.float32)
-    w_dev = torch.from_numpy(w32).cuda()
-    out = layer.forward(x, ids_dev, w_dev, offsets, sorted_slot, slot_pos)
-    torch.cuda.synchronize()
-    got = bf16_to_f64(out)
-    toks = sample_tokens(T, ids_o, n_float_tokens or T)
-    ref = lay.moe_tokens(toks, ids_o, w32.astype(np.float64), threads=host_threads())
-    rel, mabs = assert_close(got[toks], ref, f"{wl.name} out")
-    # --- end to end (GPU routing) on tokens whose routing is unambiguous ------
-    out2 = layer(x, bias, tok, tab)
-    torch.cuda.synchronize()
-    got2 = bf16_to_f64(out2)
-    e2e = toks[ok[toks]]
-    if e2e.size:
-        assert_close(got2[e2e], ref[ok[toks]], f"{wl.name} end-to-end")
-    # routing outputs of the whole-layer call (small batches route inside the
-    # fused decode kernel): ids / weights as the oracle's, permutation exact
-    import mxfp4_routed_expert_v4moe_b200 as V
-    assert V.v4moe_read_device_status(layer.workspace(T)) == V.V4MOE_OK
-    b = layer.buffers(T)
-    ids_l = b["topk_ids"].cpu().numpy()
-    w_l = b["topk_w"].cpu().numpy().astype(np.float64)
-    assert np.array_equal(ids_l[ok], ids_o[ok]), "whole-layer ids differ on non-tie tokens"
-    if ok.any():
-        assert_close(w_l[ok], w_o[ok], "whole-layer topk_w")
-    c_l, off_l, ss_l, sp_l = O.permute(ids_l, wl.E)
-    assert np.array_equal(b["counts"].cpu().numpy(), c_l)
-    assert np.array_equal(b["offsets"].cpu().numpy(), off_l)
-    assert np.array_equal(b["sorted_slot"].cpu().numpy()[:S], ss_l)
-    assert np.array_equal(b["slot_pos"].cpu().numpy()[:S], sp_l)
-    if report is not None:
-        report.update(near_ties=int(near.sum()), rel_l2=rel, max_abs=mabs, tokens=len(toks))
-    return got, ref
 
 
 def test_tiny_layer_all_tokens():
@@ -184,9 +121,15 @@ def test_bad_ids_flagged_not_faulting():
 
 
 @pytest.mark.parametrize("name,n_tok", [("decode_b1", None), ("decode_b64", None),
-                                        ("prefill_4096", 48), ("hash_16384", 48)])
+                                        ("prefill_1024", 256), ("prefill_4096", 256),
+                                        ("hash_16384", 256)])
 def test_full_size_workloads(name, n_tok, full_weights):
-    wl = IN.WORKLOADS[name]
+    """The five workloads at full size, plus a 1024-token prefill chunk whose
+    experts average 24 slots (the weight-major block-scaled GEMM with 128-slot
+    token tiles, and the shared expert's f16 GEMM). Float outputs on 256
+    sampled tokens for the large batches, always including tokens of the
+    hottest expert."""
+    wl = IN.WORKLOADS[name] if name in IN.WORKLOADS else IN.WORKLOADS["prefill_4096"].replace(name=name, T=1024)
     li = IN.make_layer_inputs(wl, weights=full_weights)
     rep = {}
     run_parity(li, _layer(li), n_float_tokens=n_tok, report=rep)

@@ -15,17 +15,17 @@ def _ids(T, k, E, seed):
     rng = np.random.default_rng(seed)
     ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
     ids[: T // 3, 0] = 5  # a hot expert
-    return ids
+    return ids.reshape(T, k)
 
 
 def _run(V, cfg, ids, static):
     T, k = ids.shape
     E = cfg.n_experts
-    d = torch.from_numpy(ids).cuda()
+    d = torch.from_numpy(np.ascontiguousarray(ids)).cuda()
     counts = torch.full((E,), -7, dtype=torch.int32, device="cuda")
     offsets = torch.full((E + 1,), -7, dtype=torch.int32, device="cuda")
-    ss = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
-    sp = torch.full((T * k,), -7, dtype=torch.int32, device="cuda")
+    ss = torch.full((max(T * k, 1),), -7, dtype=torch.int32, device="cuda")
+    sp = torch.full((max(T * k, 1),), -7, dtype=torch.int32, device="cuda")
     if static:
         rc = V.v4moe_permute_static(cfg, T, d, counts, offsets, ss, sp)
     else:
@@ -37,17 +37,23 @@ def _run(V, cfg, ids, static):
     return [t.cpu().numpy() for t in (counts, offsets, ss, sp)]
 
 
-def test_static_scratch_permute_matches_workspace_permute_twice():
+def test_static_scratch_permute_matches_workspace_permute_call_after_call():
     import mxfp4_routed_expert_v4moe_b200 as V
     cfg = V.make_config(4096, 2048, 256, 6, 2048)
-    # first call: many chunks (multi-CTA path); second call: one CTA path and
-    # smaller sizes, so stale contents from the first call would show
-    for T, seed in ((9000, 1), (37, 2)):
-        ids = _ids(T, 6, 256, seed)
+    bad = _ids(300, 6, 256, 3)
+    bad[17, 2] = 256      # out of range: skipped by both entry points
+    bad[40, 0] = -3
+    # Both multi-chunk calls use the shared chunk tables with different chunk
+    # counts (27, then 15), so stale contents from one call would show in the
+    # next; then the single-CTA path, an empty batch, and bad ids.
+    for ids in (_ids(9000, 6, 256, 1), _ids(5000, 6, 256, 2), _ids(37, 6, 256, 4),
+                np.zeros((0, 6), np.int32), bad, _ids(9000, 6, 256, 5)):
         want = _run(V, cfg, ids, static=False)
         got = _run(V, cfg, ids, static=True)
         for a, b in zip(got, want):
             assert np.array_equal(a, b)
-    # sizes beyond the fixed array are refused before any launch
-    big = V.make_config(4096, 2048, 256, 6, 2048)
-    assert V.v4moe_permute_static(big, 65536 // 6 + 1, 16, 16, 16, 16, 16) == V.V4MOE_ERR_INVALID_ARG
+    # sizes beyond the fixed array, and configs v4moe_permute refuses, are
+    # refused before any launch
+    assert V.v4moe_permute_static(cfg, 65536 // 6 + 1, 16, 16, 16, 16, 16) == V.V4MOE_ERR_INVALID_ARG
+    odd = V.make_config(4096, 2048 + 64, 256, 6, 2048)   # inter not a multiple of 128
+    assert V.v4moe_permute_static(odd, 4, 16, 16, 16, 16, 16) == V.V4MOE_ERR_INVALID_ARG
