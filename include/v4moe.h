@@ -34,8 +34,12 @@
  *    in a state the next call accepts; v4moe_clear_device_status restores
  *    them). Those bytes hold a device status word that kernels set when they
  *    meet bad data (an out-of-range expert or token id, which they skip) or
- *    give up a bounded wait; read it with v4moe_read_device_status. Calls
- *    that share a workspace must not overlap on the GPU.
+ *    give up a bounded wait; read it with v4moe_read_device_status. Word 1
+ *    of the block is a test hook of the decode path (T <= 8): when non-zero,
+ *    the router's wait inside the kernel can never be met and gives up after
+ *    that many polls (status V4MOE_ERR_TIMEOUT); zero (the default, and what
+ *    v4moe_clear_device_status writes) disarms it. Calls that share a
+ *    workspace must not overlap on the GPU.
  *  - Return value: a V4MOE_* status code. Argument errors are detected on the
  *    host before anything is launched; data errors are visible only through
  *    the device status word.
@@ -181,10 +185,9 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x,
 
 /* The whole layer in one call: v4moe_route, v4moe_permute and v4moe_forward
  * with the same arguments and results (routing outputs included). For small
- * batches (T <= 8) routing, permutation and the activation layout run as a
- * single fused kernel (its last CTA does the selection and the sort), and the
- * expert kernels stream the shared expert's weights while routing is still
- * being computed. */
+ * batches (T <= 8) the whole layer is one persistent kernel: every CTA scores
+ * its share of the experts and then selects each token's experts from all
+ * the scores, while it already streams the shared expert's weights. */
 int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const void* gate,
                     const float* bias, const int32_t* token_ids, const int32_t* tid2eid,
                     const v4moe_weights* weights, int32_t* topk_ids, float* topk_w,

@@ -42,10 +42,11 @@ int route_ksplit(const v4moe_config& c, int64_t T);
 constexpr int kShMinTokens = 512;
 size_t sh_extra_bytes(const v4moe_config& c, int64_t T);
 
-// Buffers of the decode path (all zero bytes when T is above its limit). ctl
-// holds the routing tables and a ticket that is zero at rest.
+// Buffers of the decode path (all zero bytes when T is above its limit): ctl
+// holds counters that are zero at rest, dh the intermediates, part the w2
+// partial sums per expert.
 struct DecodeBuffers {
-  size_t ctl = 0, dh = 0, hs = 0;
+  size_t ctl = 0, dh = 0, part = 0;
 };
 DecodeBuffers dec_buffers(const v4moe_config& c, int64_t T);
 
@@ -63,7 +64,7 @@ struct WsLayout {
   size_t sigma = 0;         // [T] int32 per-token power-of-two exponents
   size_t tc = 0;            // tensor-core path: activations in slot order + tile lists
   size_t sh16 = 0;          // shared expert weights widened to f16 (large batches)
-  size_t d_ctl = 0, d_dh = 0, d_hs = 0;  // decode path
+  size_t d_ctl = 0, d_dh = 0, d_part = 0;  // decode path
   size_t total = 0;
   int nchunks = 0;
 };
@@ -94,7 +95,7 @@ inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
   const DecodeBuffers d = dec_buffers(c, T);
   L.d_ctl = take(d.ctl);
   L.d_dh = take(d.dh);
-  L.d_hs = take(d.hs);
+  L.d_part = take(d.part);
   L.total = off;
   return L;
 }
@@ -178,9 +179,8 @@ cudaError_t launch_linear_w8a16(int T, int G, int N, int K, const __nv_bfloat16*
 cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, char* sh16,
                               cudaStream_t st);
 
-// Decode path: the whole layer (routing included in layer mode) as three
-// kernels chained by programmatic dependent launch, for at most
-// kDecodeMaxTokens tokens.
+// Decode path: the whole layer (routing included in layer mode) in one
+// persistent kernel, for at most kDecodeMaxTokens tokens.
 constexpr int kDecodeMaxTokens = 8;
 struct DecodeArgs {
   v4moe_config c;
@@ -203,9 +203,9 @@ struct DecodeArgs {
   uint32_t* status;
   uint32_t* ctl;
   __half* dh;
-  __half* hs;
+  float* part;
 };
-bool dec_supported(const v4moe_config& c, int T);
+bool dec_supported(const v4moe_config& c, int T, const v4moe_weights& w);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- device helpers
