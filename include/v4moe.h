@@ -36,8 +36,9 @@
  *    meet bad data (an out-of-range expert or token id, which they skip) or
  *    give up a bounded wait; read it with v4moe_read_device_status. Word 1
  *    of the block is a test hook of the decode path (T <= 8): when non-zero,
- *    the router's wait inside the kernel can never be met and gives up after
- *    that many polls (status V4MOE_ERR_TIMEOUT); zero (the default, and what
+ *    the expert kernel first waits on a barrier that nothing arrives at,
+ *    gives up after that many polls (status V4MOE_ERR_TIMEOUT) and returns
+ *    without computing; zero (the default, and what
  *    v4moe_clear_device_status writes) disarms it. Calls that share a
  *    workspace must not overlap on the GPU.
  *  - Return value: a V4MOE_* status code. Argument errors are detected on the
@@ -185,9 +186,10 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x,
 
 /* The whole layer in one call: v4moe_route, v4moe_permute and v4moe_forward
  * with the same arguments and results (routing outputs included). For small
- * batches (T <= 8) the whole layer is one persistent kernel: every CTA scores
- * its share of the experts and then selects each token's experts from all
- * the scores, while it already streams the shared expert's weights. */
+ * batches (T <= 8) the router scores run in one small kernel and the expert
+ * kernels, chained to it by programmatic dependent launch, select each
+ * token's experts themselves while they already stream the shared expert's
+ * weights. */
 int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const void* gate,
                     const float* bias, const int32_t* token_ids, const int32_t* tid2eid,
                     const v4moe_weights* weights, int32_t* topk_ids, float* topk_w,

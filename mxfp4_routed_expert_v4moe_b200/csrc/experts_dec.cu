@@ -1,0 +1,1180 @@
+// Decode-sized batches (at most 8 tokens): the layer as three kernels chained
+// by programmatic dependent launch, streaming every weight byte once.
+//
+// What it computes ("Checked in its code" rows "Mixture of experts",
+// "Auxiliary-loss-free load balancing", "SwiGLU feed-forward", "Shared
+// expert"; "config.json" experts_w4a16 / linears_w8a16):
+//   layer mode: s[t, e] = sqrt(softplus(gate[e] . x_t)), top-k of s + bias (or
+//   the token-id hash table), w = scale * s / sum; forward mode takes ids and
+//   weights from the caller. Then, for the shared expert and every routed
+//   expert the batch hits,
+//     h = silu(min(g, L)) * clamp(u, -L, L),   [g; u] = W13 x_t,
+//     out_t = W2_shared hs_t + sum over the token's experts of w * W2_e h.
+//
+// Kernels:
+//  * k_dec_route: router scores (one warp per expert); the last CTA to finish
+//    selects each token's experts and publishes the batch's routing tables
+//    (distinct experts in ascending id, token masks, weights) and the
+//    permutation outputs. In forward mode one CTA publishes the tables of the
+//    caller's routing.
+//  * k_dec_w13: one CTA per SM, two groups of eight warps. Work items are w13
+//    slabs (8 channels of a routed expert: 8 gate rows and the 8 matching up
+//    rows; or 4 + 4 int8 rows of the shared expert), numbered shared first,
+//    then routed expert by expert; CTA b takes a contiguous share of each as
+//    its ring positions 0, 1, .... The shared slabs do not depend on the
+//    routing: their copies are issued at the start and group 1 multiplies
+//    them while group 0 selects from the router's scores and builds the
+//    routing tables; then both groups take alternate positions of the routed
+//    slabs, and once its last slab is on its way the CTA asks L2 for its
+//    share of the routed w2 rows. Warp i of a group owns the 128-wide K
+//    blocks i, i + 8, ... of a slab, multiplies them by the activations with
+//    mma.sync m16n8k16 (f16 operands, fp32 accumulation, the tokens as the 8
+//    columns) and posts its partial tile to shared memory; the last warp to
+//    post sums the partials in warp order, refills the stage and writes h as
+//    f16 (routed: w * h).
+//  * k_dec_w2: two groups of eight warps, warp i of a group owning K blocks
+//    i, i + 8. CTA b owns a run of 16-row output blocks and goes through the
+//    shared expert and every routed expert for each of them, the two groups
+//    taking alternate experts; a stage holds
+//    the expert's 16 weight rows and the intermediates of its tokens. The sum
+//    over experts (shared first, then ascending id) is formed in registers and
+//    written once as bf16, so the result does not depend on timing.
+//
+// The intermediates are stored as f16 scaled by a fixed power of two chosen
+// from the clamp limit: |h| <= L * L * routed_scale, so h * 2^tau stays below
+// the f16 maximum for every input while small values keep that many more
+// binades; the down projection divides it out.
+//
+// Operands are exact: E2M1 pairs via cvt.rn.f16x2.e2m1x2, int8 via a
+// magic-number conversion; the E8M0 group scale multiplies the f16 operand as
+// a power of two relative to the largest exponent among the warp's groups of
+// that row, and the rest is applied in fp32. Activations are f16, scaled per
+// token by a power of two that puts the row maximum in [2^14, 2^15).
+//
+// No CTA waits on another CTA: data crosses kernels only at the programmatic
+// launch boundaries (griddepcontrol.wait), which also order memory. Every
+// mbarrier wait is bounded and flags the status word.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "launch.cuh"
+#include "ptx.cuh"
+#include "route_dev.cuh"
+#include "v4moe_internal.cuh"
+
+namespace v4moe {
+namespace {
+
+constexpr int kGW = 8;             // warps per consumer group (w13 kernel)
+constexpr int kThreads = 16 * 32;  // both slab kernels
+constexpr int kStages13 = 5;
+constexpr int kMaxStages2 = 6;
+constexpr int kNJ = 4;             // K blocks per warp held in registers (K <= 4096)
+constexpr int kMaxHit = 64;        // distinct routed experts of a batch (T * k <= 64)
+constexpr int kShRows = 64;        // shared-expert rows per CTA with preloaded scales
+constexpr uint32_t kBarTries = 1u << 20;
+
+// Control block words (workspace): the routing tables, rewritten by every
+// call for the w2 kernel.
+enum Ctl : int {
+  cNh = 0,
+  cHit = 32,          // [kMaxHit] expert id per list index
+  cMask = cHit + 64,  // [kMaxHit] bit per token routed to the expert
+  cW = cMask + 64,    // [kMaxHit][8] float weight per (expert, token)
+  cWords = cW + 64 * 8,
+};
+
+struct DecParams {
+  int T, H, I, Is, E, k, vocab;
+  float limit, routed_scale;
+  float tau_r, tau_s;  // the intermediates are stored as f16(h * tau): routed, shared
+  int layer_mode;
+  int stage_bytes;
+  int nstages;  // w2 ring depth
+  int w2_per;   // 16-row output blocks per w2 CTA
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* gate;
+  const float* bias;
+  const int32_t* token_ids;
+  const int32_t* tid2eid;
+  int32_t* topk_ids;  // layer mode: written; forward mode: read
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_slot;
+  int32_t* slot_pos;
+  float* scores;  // [T, E]
+  const uint8_t* w13_codes;
+  const uint8_t* w13_scales;
+  const uint8_t* w2_codes;
+  const uint8_t* w2_scales;
+  const int8_t* sh13;
+  const float* sh13_scale;
+  const int8_t* sh2;
+  const float* sh2_scale;
+  __half* dh;  // [kMaxHit, T, I] weighted routed intermediates
+  __half* hs;  // [T, Is] shared intermediates
+  uint32_t* ctl;
+  uint32_t* status;
+  __nv_bfloat16* out;
+};
+
+// Routing tables as the slab kernels keep them in shared memory.
+struct Tables {
+  int nh;
+  int hit[kMaxHit];
+  uint32_t mask[kMaxHit];
+  float w[kMaxHit * 8];
+};
+
+__device__ __forceinline__ float pow2f(int e) {
+  e = max(-126, min(127, e));
+  return __int_as_float((e + 127) << 23);
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const DecParams& P) {
+  if (mbar_wait_bounded(bar, parity, kBarTries)) return true;
+  atomicOr(P.status, kStatusTimeout);
+  return false;
+}
+
+// 14 - floor(log2 m) for the largest bf16 magnitude bits m of a row (0 for an
+// all-zero row), clamped to [-120, 120]: 2^sigma * max lies in [2^14, 2^15).
+__device__ __forceinline__ int sigma_of(uint32_t mx) {
+  if (mx == 0) return 0;
+  const int ef = int(mx >> 7);
+  const int sg = ef == 0 ? 120 : 141 - ef;
+  return max(-120, min(120, sg));
+}
+
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t w) {
+  return max(m, max(w & 0x7FFFu, (w >> 16) & 0x7FFFu));
+}
+
+// Whole CTA; the caller synchronises afterwards.
+__device__ __forceinline__ void read_tables(Tables& tb, const DecParams& P) {
+  const int nh = int(P.ctl[cNh]);
+  for (int i = threadIdx.x; i < nh; i += blockDim.x) {
+    tb.hit[i] = int(P.ctl[cHit + i]);
+    tb.mask[i] = P.ctl[cMask + i];
+  }
+  for (int i = threadIdx.x; i < nh * 8; i += blockDim.x) tb.w[i] = reinterpret_cast<const float*>(P.ctl + cW)[i];
+  if (threadIdx.x == 0) tb.nh = nh;
+}
+
+// ---------------------------------------------------------------- slab products
+
+// MXFP4 m16 tile: rows g and g + 8 of the tile at ra / rb (codes of 128-wide
+// K block kb at kb * 64), their E8M0 scale rows at sa / sb. The warp's K
+// blocks kb = wi + KS j (j < NJ, kb < nkb) multiply B[j]. Even and odd MMA
+// steps go to separate accumulators; fa / fb get the fp32 factors of the two
+// rows.
+template <int NJ, int KS>
+__device__ __forceinline__ void tile_mx(const char* ra, const char* rb, const uint8_t* sa, const uint8_t* sb, int wi,
+                                        int nkb, const uint32_t (&B)[NJ][16], float (&ae)[4], float (&ao)[4],
+                                        float& fa, float& fb) {
+  const int t = threadIdx.x & 3;
+  int xa = 0, xb = 0;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int kb = wi + KS * j;
+    if (kb < nkb) {
+      xa = max(xa, int(sa[4 * kb + t]));
+      xb = max(xb, int(sb[4 * kb + t]));
+    }
+  }
+  xa = max(xa, __shfl_xor_sync(0xffffffffu, xa, 1));
+  xa = max(xa, __shfl_xor_sync(0xffffffffu, xa, 2));
+  xb = max(xb, __shfl_xor_sync(0xffffffffu, xb, 1));
+  xb = max(xb, __shfl_xor_sync(0xffffffffu, xb, 2));
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int kb = wi + KS * j;
+    if (kb < nkb) {
+      const uint4 qa = *reinterpret_cast<const uint4*>(ra + kb * 64 + 16 * t);
+      const uint4 qb = *reinterpret_cast<const uint4*>(rb + kb * 64 + 16 * t);
+      const uint32_t fsa = f16_pow2_bits(int(sa[4 * kb + t]) - xa + 13) * 0x10001u;
+      const uint32_t fsb = f16_pow2_bits(int(sb[4 * kb + t]) - xb + 13) * 0x10001u;
+      const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
+      const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t ca[4], cb[4];
+        e2m1x8_to_f16x2(wa[u], ca);
+        e2m1x8_to_f16x2(wb[u], cb);
+        const uint32_t A0[4] = {hmul2_u32(ca[0], fsa), hmul2_u32(cb[0], fsb), hmul2_u32(ca[1], fsa),
+                                hmul2_u32(cb[1], fsb)};
+        const uint32_t A1[4] = {hmul2_u32(ca[2], fsa), hmul2_u32(cb[2], fsb), hmul2_u32(ca[3], fsa),
+                                hmul2_u32(cb[3], fsb)};
+        mma_16816_f16(ae, A0, B[j][4 * u], B[j][4 * u + 1]);
+        mma_16816_f16(ao, A1, B[j][4 * u + 2], B[j][4 * u + 3]);
+      }
+    }
+  }
+  fa = pow2f(xa - 127 - 13);
+  fb = pow2f(xb - 127 - 13);
+}
+
+// int8 m16 tile: rows g and g + 8 at ra / rb (K block kb at (kb - kb0) * 128),
+// zero rows where `valid` is false. The warp's K blocks kb = wi + KS j inside
+// [kb0, kb1) multiply B[j].
+template <int NJ, int KS>
+__device__ __forceinline__ void tile_s8(const char* ra, const char* rb, bool valid, int kb0, int kb1, int wi,
+                                        const uint32_t (&B)[NJ][16], float (&ae)[4], float (&ao)[4]) {
+  const int t = threadIdx.x & 3;
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int kb = wi + KS * j;
+    if (kb >= kb0 && kb < kb1) {
+      uint4 qa0 = make_uint4(0u, 0u, 0u, 0u), qa1 = qa0, qb0 = qa0, qb1 = qa0;
+      if (valid) {
+        const char* pa = ra + (kb - kb0) * 128 + 32 * t;
+        const char* pb = rb + (kb - kb0) * 128 + 32 * t;
+        qa0 = *reinterpret_cast<const uint4*>(pa);
+        qa1 = *reinterpret_cast<const uint4*>(pa + 16);
+        qb0 = *reinterpret_cast<const uint4*>(pb);
+        qb1 = *reinterpret_cast<const uint4*>(pb + 16);
+      }
+      const uint32_t wa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
+      const uint32_t wb[8] = {qb0.x, qb0.y, qb0.z, qb0.w, qb1.x, qb1.y, qb1.z, qb1.w};
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        uint32_t A[4];
+        s8x4_to_f16x2(wa[s], A[0], A[2]);
+        s8x4_to_f16x2(wb[s], A[1], A[3]);
+        if (s & 1)
+          mma_16816_f16(ao, A, B[j][2 * s], B[j][2 * s + 1]);
+        else
+          mma_16816_f16(ae, A, B[j][2 * s], B[j][2 * s + 1]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- routing
+
+// Selection and routing tables, built in shared memory by every w13 CTA.
+struct RouteSmem {
+  uint32_t bits[32];
+  int rank_base[32];
+  int cnt[kMaxHit];
+  int cum[kMaxHit + 1];
+  int ids[64];
+  float wts[64];
+  int32_t sel_ids[64];  // the selection's output
+  float sel_w[64];
+};
+
+// The batch's routed experts in ascending id, per (expert, token) weights and
+// token masks, from topk ids / weights (global or shared memory), into tb;
+// one warp. Out-of-range ids are skipped and, unless `quiet`, flagged.
+__device__ __forceinline__ void route_tables(RouteSmem& S, Tables& tb, const DecParams& P, const int32_t* tids,
+                                             const float* tw, bool quiet) {
+  const int lane = threadIdx.x & 31;
+  const int Sn = P.T * P.k;
+  S.bits[lane] = 0u;
+  __syncwarp();
+  bool bad = false;
+  for (int s = lane; s < 64; s += 32) {
+    int e = -1;
+    float w = 0.f;
+    if (s < Sn) {
+      e = tids[s];
+      w = tw[s];
+      if (e < 0 || e >= P.E) {
+        bad = true;
+        e = -1;
+      }
+    }
+    S.ids[s] = e;
+    S.wts[s] = w;
+    if (e >= 0) atomicOr(&S.bits[e >> 5], 1u << (e & 31));
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && !quiet) atomicOr(P.status, kStatusBadExpertId);
+  __syncwarp();
+  const uint32_t word = S.bits[lane];
+  const int c = __popc(word);
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  S.rank_base[lane] = incl - c;
+  const int nh = __shfl_sync(0xffffffffu, incl, 31);
+  for (int i = lane; i < kMaxHit * 8; i += 32) tb.w[i] = 0.f;
+  for (int i = lane; i < kMaxHit; i += 32) {
+    tb.mask[i] = 0u;
+    S.cnt[i] = 0;
+  }
+  __syncwarp();
+  for (int s = lane; s < Sn; s += 32) {
+    const int e = S.ids[s];
+    if (e >= 0) {
+      const int r = S.rank_base[e >> 5] + __popc(S.bits[e >> 5] & ((1u << (e & 31)) - 1u));
+      const int tok = s / P.k;
+      tb.hit[r] = e;
+      atomicAdd(&tb.w[r * 8 + tok], S.wts[s]);
+      atomicOr(&tb.mask[r], 1u << tok);
+      atomicAdd(&S.cnt[r], 1);
+    }
+  }
+  if (lane == 0) tb.nh = nh;
+  __syncwarp();
+}
+
+// The tables, for the w2 kernel (one warp).
+__device__ __noinline__ void publish_tables(const Tables& tb, const DecParams& P) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < tb.nh; i += 32) {
+    P.ctl[cHit + i] = uint32_t(tb.hit[i]);
+    P.ctl[cMask + i] = tb.mask[i];
+  }
+  for (int i = lane; i < tb.nh * 8; i += 32) reinterpret_cast<float*>(P.ctl + cW)[i] = tb.w[i];
+  if (lane == 0) P.ctl[cNh] = uint32_t(tb.nh);
+}
+
+// Stable counting sort of the batch's slots by expert (layer-mode outputs),
+// from the state route_tables left in shared memory; one warp.
+__device__ __noinline__ void write_permutation(RouteSmem& S, const DecParams& P, int nh) {
+  const int lane = threadIdx.x & 31;
+  const int Sn = P.T * P.k;
+  const int c0 = 2 * lane < nh ? S.cnt[2 * lane] : 0;
+  const int c1 = 2 * lane + 1 < nh ? S.cnt[2 * lane + 1] : 0;
+  int incl = c0 + c1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  const int excl = incl - c0 - c1;
+  S.cum[2 * lane] = excl;
+  S.cum[2 * lane + 1] = excl + c0;
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (lane == 0) S.cum[kMaxHit] = total;
+  __syncwarp();
+  for (int e = lane; e < P.E; e += 32) {
+    const uint32_t word = S.bits[e >> 5];
+    const int r = S.rank_base[e >> 5] + __popc(word & ((1u << (e & 31)) - 1u));
+    const bool hit = (word >> (e & 31)) & 1u;
+    P.counts[e] = hit ? S.cnt[r] : 0;
+    P.offsets[e] = r < nh ? S.cum[r] : total;
+  }
+  if (lane == 0) P.offsets[P.E] = total;
+  for (int s = lane; s < Sn; s += 32) {
+    const int e = S.ids[s];
+    if (e < 0) continue;
+    const int r = S.rank_base[e >> 5] + __popc(S.bits[e >> 5] & ((1u << (e & 31)) - 1u));
+    int before = 0;
+    for (int s2 = 0; s2 < s; ++s2) before += S.ids[s2] == e;
+    const int pos = S.cum[r] + before;
+    P.sorted_slot[pos] = s;
+    P.slot_pos[s] = pos;
+  }
+}
+
+// Top-k selection of token t (one warp) from scores and bias in shared memory,
+// into the RouteSmem selection arrays. Inlined: the routing runs while the
+// shared slabs' copies are in flight, and on this GPU the local-memory traffic
+// of a call (saved registers) would wait behind them.
+__device__ __forceinline__ void select_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
+                                             const float* sbias) {
+  if (P.token_ids)
+    select_hash_warp<true>(t, P.E, P.k, P.vocab, P.routed_scale, ssc + size_t(t) * P.E, P.token_ids, P.tid2eid,
+                           S.sel_ids, S.sel_w, P.status);
+  else if (P.E <= 256)
+    select_learned_n<false, 8>(t, P.E, P.k, P.routed_scale, ssc + size_t(t) * P.E, sbias, S.sel_ids, S.sel_w);
+  else
+    select_learned_n<false, 32>(t, P.E, P.k, P.routed_scale, ssc + size_t(t) * P.E, sbias, S.sel_ids, S.sel_w);
+}
+
+constexpr int kRouteWarps = 8;
+
+// Router scores s[t, e] (one warp per expert, the x rows staged in shared
+// memory). The selection happens in every CTA of the next kernel.
+__global__ void __launch_bounds__(kRouteWarps * 32) k_dec_route(DecParams P) {
+  extern __shared__ __align__(16) char rsm[];
+  // The w13 kernel may start now: before it waits for this grid it only reads
+  // the activations and asks L2 for weights.
+  pdl_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = P.H, T = P.T, E = P.E;
+  uint4* xs = reinterpret_cast<uint4*>(rsm);
+  const int e = blockIdx.x * kRouteWarps + warp;
+  // the whole gate row in flight at once (H <= 4096: up to 16 pieces per lane)
+  const uint4* grow = reinterpret_cast<const uint4*>(P.gate + size_t(e < E ? e : 0) * H);
+  const int np = H / 8 / 32;
+  uint4 gv[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) gv[i] = i < np ? __ldg(grow + lane + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
+  for (int i = threadIdx.x; i < T * H / 8; i += blockDim.x) xs[i] = __ldg(reinterpret_cast<const uint4*>(P.x) + i);
+  __syncthreads();
+  if (e >= E) return;
+  for (int t = 0; t < T; ++t) {
+    const uint4* xrow = xs + size_t(t) * (H / 8);
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < np) {
+        const uint4 xv = xrow[lane + 32 * i];
+        acc = fmaf(bf16_lo(gv[i].x), bf16_lo(xv.x), acc);
+        acc = fmaf(bf16_hi(gv[i].x), bf16_hi(xv.x), acc);
+        acc = fmaf(bf16_lo(gv[i].y), bf16_lo(xv.y), acc);
+        acc = fmaf(bf16_hi(gv[i].y), bf16_hi(xv.y), acc);
+        acc = fmaf(bf16_lo(gv[i].z), bf16_lo(xv.z), acc);
+        acc = fmaf(bf16_hi(gv[i].z), bf16_hi(xv.z), acc);
+        acc = fmaf(bf16_lo(gv[i].w), bf16_lo(xv.w), acc);
+        acc = fmaf(bf16_hi(gv[i].w), bf16_hi(xv.w), acc);
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) P.scores[size_t(t) * E + e] = sqrt_softplus_f(acc);
+  }
+}
+
+// ---------------------------------------------------------------- w13 kernel
+
+struct W13Smem {
+  uint64_t full[kStages13];
+  int redcnt[kStages13];
+  int lastfill[kStages13];
+  int sigma[2][8];  // per consumer group
+  uint32_t xmax[2][kGW][8];
+  float sh_scale[2][kShRows];  // gate / up row scales of this CTA's shared slabs
+  Tables tb;
+  RouteSmem rt;
+  int ready;          // group 0 has built the tables
+};
+
+constexpr size_t kHead13 = (sizeof(W13Smem) + 127) / 128 * 128;
+constexpr size_t kPart13 = size_t(kStages13) * kGW * 32 * 16;  // float4 per lane and warp
+
+enum Kind : int { kEnd = 0, kS13 = 1, kR13 = 2 };
+struct Item {
+  int kind, li, row0, e;
+};
+
+// Item number -> slab: shared w13 slabs (4 gate + 4 up int8 rows) first, then
+// routed w13 slabs (8 + 8 MXFP4 rows), expert by expert.
+__device__ __forceinline__ Item w13_item(const DecParams& P, const Tables& tb, int it) {
+  Item m = {kEnd, 0, 0, 0};
+  const int n_s = P.Is > 0 ? P.Is / 4 : 0;
+  if (it < n_s) {
+    m.kind = kS13;
+    m.row0 = it * 4;
+  } else {
+    const int r = it - n_s, i8 = P.I / 8;
+    if (r < tb.nh * i8) {
+      m.kind = kR13;
+      m.li = r / i8;
+      m.row0 = (r % i8) * 8;
+      m.e = tb.hit[m.li];
+    }
+  }
+  return m;
+}
+
+// Copies slab m into stage s (lane 0 of the calling warp issues and arms).
+__device__ __forceinline__ void fill13(const DecParams& P, W13Smem& S, char* dst, int s, const Item& m, int pos) {
+  const int H = P.H;
+  if ((threadIdx.x & 31) == 0) {
+    S.lastfill[s] = pos;
+    if (m.kind == kS13) {
+      const char* sh = reinterpret_cast<const char*>(P.sh13);
+      mbar_arrive_expect_tx(&S.full[s], uint32_t(8 * H));
+      bulk_g2s(dst, sh + size_t(m.row0) * H, uint32_t(4 * H), &S.full[s]);
+      bulk_g2s(dst + 4 * H, sh + size_t(P.Is + m.row0) * H, uint32_t(4 * H), &S.full[s]);
+    } else {
+      const size_t rg = size_t(m.e) * 2 * P.I + m.row0, ru = rg + P.I;
+      mbar_arrive_expect_tx(&S.full[s], uint32_t(16 * (H / 2) + 16 * (H / 32)));
+      bulk_g2s(dst, P.w13_codes + rg * (H / 2), uint32_t(8 * (H / 2)), &S.full[s]);
+      bulk_g2s(dst + 8 * (H / 2), P.w13_codes + ru * (H / 2), uint32_t(8 * (H / 2)), &S.full[s]);
+      bulk_g2s(dst + 16 * (H / 2), P.w13_scales + rg * (H / 32), uint32_t(8 * (H / 32)), &S.full[s]);
+      bulk_g2s(dst + 16 * (H / 2) + 8 * (H / 32), P.w13_scales + ru * (H / 32), uint32_t(8 * (H / 32)),
+               &S.full[s]);
+    }
+  }
+  __syncwarp();
+}
+
+// CTA b's share of the w13 slabs: shared slabs [s0, s1) and routed slabs
+// [r0, r1) (routed slab r is item n_s + r), contiguous so that each expert's
+// rows form one range per CTA. Ring position p is the p-th of these.
+struct Chunk {
+  int s0, s1, r0, r1;
+  __device__ int size() const { return (s1 - s0) + (r1 - r0); }
+  __device__ int item(int p, int n_s) const { return p < s1 - s0 ? s0 + p : n_s + r0 + (p - (s1 - s0)); }
+};
+__device__ __forceinline__ Chunk w13_chunk(const DecParams& P, int nh, int b, int G) {
+  Chunk c;
+  const int n_s = P.Is > 0 ? P.Is / 4 : 0, n_r = nh * (P.I / 8);
+  const int per_s = (n_s + G - 1) / G, per_r = (n_r + G - 1) / G;
+  c.s0 = min(n_s, b * per_s);
+  c.s1 = min(n_s, c.s0 + per_s);
+  c.r0 = min(n_r, b * per_r);
+  c.r1 = min(n_r, c.r0 + per_r);
+  return c;
+}
+
+// The w2 rows of the 16-row output blocks that CTA b of the w2 kernel owns
+// (blocks [b w2_per, (b + 1) w2_per)): the shared expert's, or every routed
+// expert's (one lane).
+__device__ __forceinline__ void prefetch_w2_share(const DecParams& P, const Tables& tb, int b, bool routed) {
+  const int nrb = P.H / 16;
+  const int rb0 = min(nrb, b * P.w2_per), rb1 = min(nrb, rb0 + P.w2_per);
+  if (rb1 <= rb0) return;
+  const size_t rows = size_t(16) * (rb1 - rb0);
+  if (!routed) {
+    if (P.Is > 0) prefetch_l2_range(reinterpret_cast<const char*>(P.sh2) + size_t(16 * rb0) * P.Is, rows * P.Is);
+    return;
+  }
+  for (int li = 0; li < tb.nh; ++li) {
+    const size_t r0 = size_t(tb.hit[li]) * P.H + size_t(16) * rb0;
+    prefetch_l2_range(P.w2_codes + r0 * (P.I / 2), rows * (P.I / 2));
+    prefetch_l2_range(P.w2_scales + r0 * (P.I / 32), rows * (P.I / 32));
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
+  extern __shared__ __align__(128) char smem[];
+  W13Smem& S = *reinterpret_cast<W13Smem*>(smem);
+  // Test hook (word 1 of the status block, zero in normal use): a wait on a
+  // barrier that nothing arrives at, bounded by that many polls; it gives up,
+  // flags the timeout and the CTA returns before issuing any copy.
+  if (const uint32_t arm = __ldcg(P.status + 1)) {
+    if (threadIdx.x == 0) {
+      mbar_init(&S.full[0], 1);
+      fence_mbar_init();
+      if (!mbar_wait_bounded(&S.full[0], 0u, arm)) atomicOr(P.status, kStatusTimeout);
+    }
+    return;
+  }
+  char* stages = smem + kHead13;
+  float4* parts = reinterpret_cast<float4*>(stages + size_t(kStages13) * P.stage_bytes);
+  // router scores and bias, outside the ring (it takes the shared slabs
+  // before the routing is known)
+  float* ssc = reinterpret_cast<float*>(reinterpret_cast<char*>(parts) + kPart13);
+  float* sbias = ssc + size_t(P.T) * P.E;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = P.T, H = P.H;
+  const int G = int(gridDim.x), b = int(blockIdx.x);
+  const int n_s = P.Is > 0 ? P.Is / 4 : 0;
+  const bool learned = P.layer_mode && !P.token_ids;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages13; ++s) {
+      mbar_init(&S.full[s], 1);
+      S.redcnt[s] = 0;
+      S.lastfill[s] = -1;
+    }
+    S.tb.nh = 0;
+    S.ready = 0;
+    fence_mbar_init();
+  }
+  // The w2 kernel may launch now (its CTAs start as these leave their SMs).
+  pdl_launch_dependents();
+  // The shared range of this CTA does not depend on the routing: its first
+  // nsp slabs go into the ring before the routing is known.
+  const Chunk c0 = w13_chunk(P, 0, b, G);
+  const int nsp = min(c0.s1 - c0.s0, kStages13);
+  const int q = warp / kGW, wi = warp % kGW;
+  const int g = lane >> 2, t = lane & 3;
+  const int nkbH = H / 128;
+
+  // Global memory outside the ring is read before the first copy is issued:
+  // on this GPU a global load waits behind the SM's transfers in flight. The
+  // loads of the shared slabs' row scales and the bias (into registers,
+  // stored to shared memory after the copies are issued) and of x go out
+  // first.
+  // Group 1 (which takes the shared slabs first) loads the row scales, group
+  // 0 (which selects) the bias, so each group's own barriers order the stores
+  // before its reads.
+  constexpr int kGT = kGW * 32;  // threads per group
+  const int nsr = min(4 * (c0.s1 - c0.s0), kShRows);
+  const int gt = int(threadIdx.x) - q * kGT;  // thread within the group
+  float rsg = 0.f, rsu = 0.f, rb[4] = {0.f, 0.f, 0.f, 0.f};
+  if (q == 1 && gt < nsr) {
+    rsg = __ldg(P.sh13_scale + 4 * c0.s0 + gt);
+    rsu = __ldg(P.sh13_scale + P.Is + 4 * c0.s0 + gt);
+  }
+  if (q == 0 && learned) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (gt + j * kGT < P.E) rb[j] = __ldg(P.bias + gt + j * kGT);
+    for (int i = gt + 4 * kGT; i < P.E; i += kGT) sbias[i] = __ldg(P.bias + i);
+  }
+  // this warp's x slices (token g; in L2 after the router), loaded by each
+  // group when it is about to use them: group 1 at once, group 0 after the
+  // routing, so that the routing code runs with few live registers and no
+  // local-memory traffic (on this GPU that would wait behind the copies in
+  // flight)
+  uint32_t B[kNJ][16];
+  auto load_x = [&]() {
+  #pragma unroll
+    for (int j = 0; j < kNJ; ++j) {
+      const int kb = wi + 8 * j;
+      if (kb < nkbH && g < T) {
+        const uint4* src = reinterpret_cast<const uint4*>(P.x + size_t(g) * H + kb * 128 + 32 * t);
+  #pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const uint4 v = __ldg(src + p);
+          B[j][4 * p] = v.x;
+          B[j][4 * p + 1] = v.y;
+          B[j][4 * p + 2] = v.z;
+          B[j][4 * p + 3] = v.w;
+        }
+      } else {
+  #pragma unroll
+        for (int i = 0; i < 16; ++i) B[j][i] = 0u;
+      }
+    }
+  };
+  __syncthreads();
+  if (warp == 14)
+    for (int p = 0; p < nsp; ++p)
+      fill13(P, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, c0.s0 + p), p);
+  if (q == 1 && gt < nsr) {
+    S.sh_scale[0][gt] = rsg;
+    S.sh_scale[1][gt] = rsu;
+  }
+  if (q == 0 && learned) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (gt + j * kGT < P.E) sbias[gt + j * kGT] = rb[j];
+  }
+  // ---- f16 activations scaled by 2^sigma (each group keeps its own copy)
+  auto prep_x = [&]() {
+    load_x();
+    uint32_t mx = 0u;
+#pragma unroll
+    for (int j = 0; j < kNJ; ++j)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mx = absmax_bf16x2(mx, B[j][i]);
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if (t == 0) S.xmax[q][wi][g] = mx;
+    named_bar_sync(2 + q, kGW * 32);
+    uint32_t rmx = 0u;
+    for (int w = 0; w < kGW; ++w) rmx = max(rmx, S.xmax[q][w][g]);
+    const int sg = sigma_of(rmx);
+    if (wi == 0 && t == 0) S.sigma[q][g] = sg;
+    const float mul = __int_as_float((sg + 127) << 23);
+#pragma unroll
+    for (int j = 0; j < kNJ; ++j)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const __half2 hv = __floats2half2_rn(bf16_lo(B[j][i]) * mul, bf16_hi(B[j][i]) * mul);
+        B[j][i] = *reinterpret_cast<const uint32_t*>(&hv);
+      }
+    named_bar_sync(2 + q, kGW * 32);  // the group's sigma is visible to the group
+  };
+
+  // One slab at ring position pos (chunk ch of npos positions): the warp's K
+  // blocks, its partial tile posted to shared memory; the last warp of the
+  // group to post sums the partials in warp order, refills the stage with
+  // position pos + kStages13 when `refill`, and writes h. False after a
+  // timed-out wait.
+  auto run_item = [&](const Chunk& ch, int npos, int pos, bool refill, bool need_tables) -> bool {
+    const Item m = w13_item(P, S.tb, ch.item(pos, n_s));
+    const int s = pos % kStages13;
+    if (!__all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / kStages13) & 1u, P))) return false;
+    const char* st = stages + size_t(s) * P.stage_bytes;
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 p0;
+    if (m.kind == kR13) {
+      const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + 16 * (H / 2));
+      float fa, fb;
+      tile_mx<kNJ, 8>(st + g * (H / 2), st + (g + 8) * (H / 2), sc + g * (H / 32), sc + (g + 8) * (H / 32), wi,
+                      nkbH, B, a0, a1, fa, fb);
+      p0 = make_float4((a0[0] + a1[0]) * fa, (a0[1] + a1[1]) * fa, (a0[2] + a1[2]) * fb, (a0[3] + a1[3]) * fb);
+    } else {
+      // rows g < 4: gate row g of the slab (tile row g) and up row g (tile row g + 8)
+      tile_s8<kNJ, 8>(st + (g & 3) * H, st + (4 + (g & 3)) * H, g < 4, 0, nkbH, wi, B, a0, a1);
+      p0 = make_float4(a0[0] + a1[0], a0[1] + a1[1], a0[2] + a1[2], a0[3] + a1[3]);
+    }
+    float4* part = parts + size_t(s) * kGW * 32;
+    part[wi * 32 + lane] = p0;
+    __threadfence_block();
+    __syncwarp();
+    int old = 0;
+    if (lane == 0) old = atomicAdd(&S.redcnt[s], 1);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old != kGW - 1) return true;
+    // Last of the group: the stage and its partials are this warp's alone.
+    __threadfence_block();
+    float4 d = part[lane];
+#pragma unroll
+    for (int w = 1; w < kGW; ++w) {
+      const float4 v = part[w * 32 + lane];
+      d.x += v.x;
+      d.y += v.y;
+      d.z += v.z;
+      d.w += v.w;
+    }
+    if (lane == 0) S.redcnt[s] = 0;
+    __syncwarp();
+    if (refill) {
+      Chunk cr = ch;
+      int nr = npos;
+      bool have = true;
+      if (need_tables) {  // the next position may be routed: wait for the tables
+        uint32_t i = 0;
+        while (*reinterpret_cast<volatile int*>(&S.ready) == 0 && ++i < kBarTries) __nanosleep(32);
+        have = i < kBarTries;
+        if (!have && lane == 0) atomicOr(P.status, kStatusTimeout);
+        __threadfence_block();
+        cr = w13_chunk(P, S.tb.nh, b, G);
+        nr = cr.size();
+      }
+      if (have && pos + kStages13 < nr) {
+        fill13(P, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, cr.item(pos + kStages13, n_s)),
+               pos + kStages13);
+        if (pos + kStages13 == nr - 1 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
+      }
+      if (!have) return false;
+    }
+    const float dg[2] = {d.x, d.y}, du[2] = {d.z, d.w};
+    if (m.kind == kR13) {
+      const uint32_t mask = S.tb.mask[m.li];
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int tok = 2 * t + qq;
+        if (tok < T && ((mask >> tok) & 1u)) {
+          const float inv = pow2f(-S.sigma[q][tok]);
+          const float h = clamped_swiglu_f(dg[qq] * inv, du[qq] * inv, P.limit) * S.tb.w[m.li * 8 + tok] * P.tau_r;
+          P.dh[(size_t(m.li) * T + tok) * P.I + m.row0 + g] = __float2half_rn(h);
+        }
+      }
+    } else if (g < 4) {
+      const int rl = m.row0 + g - 4 * ch.s0;  // row within this CTA's shared slabs
+      const float sg = rl < kShRows ? S.sh_scale[0][rl] : __ldg(P.sh13_scale + m.row0 + g);
+      const float su = rl < kShRows ? S.sh_scale[1][rl] : __ldg(P.sh13_scale + P.Is + m.row0 + g);
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int tok = 2 * t + qq;
+        if (tok < T) {
+          const float inv = pow2f(-S.sigma[q][tok]);
+          P.hs[size_t(tok) * P.Is + m.row0 + g] =
+              __float2half_rn(clamped_swiglu_f(dg[qq] * sg * inv, du[qq] * su * inv, P.limit) * P.tau_s);
+        }
+      }
+    }
+    return true;
+  };
+
+  bool ok = true;
+  if (q == 1) {
+    // ---- group 1: the shared slabs already on their way, while group 0
+    // routes; their refills continue with the following positions
+    prep_x();
+    for (int pos = 0; pos < nsp && ok; ++pos) ok = run_item(c0, nsp, pos, true, true);
+  } else {
+    // ---- group 0: routing. Every CTA selects from the scores and builds the
+    // tables; the scores (previous grid) are complete and visible past the wait.
+    pdl_wait();
+    if (P.layer_mode) {
+      for (int i = threadIdx.x; i < T * P.E; i += kGT) ssc[i] = __ldcg(P.scores + i);
+      named_bar_sync(4, kGT);
+      if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
+      named_bar_sync(4, kGT);
+      if (warp == 0) route_tables(S.rt, S.tb, P, S.rt.sel_ids, S.rt.sel_w, true);
+    } else if (warp == 0) {
+      route_tables(S.rt, S.tb, P, P.topk_ids, P.topk_w, b != 0);
+    }
+    named_bar_sync(4, kGT);
+    if (warp == 0) {
+      // the stages the shared slabs did not take, then the tables are ready
+      // for group 1's refills
+      const Chunk cr = w13_chunk(P, S.tb.nh, b, G);
+      const int nr = cr.size();
+      for (int p = nsp; p < kStages13 && p < nr; ++p)
+        fill13(P, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, cr.item(p, n_s)), p);
+      if (nr <= kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
+      __threadfence_block();
+      if (lane == 0) *reinterpret_cast<volatile int*>(&S.ready) = 1;
+    }
+    if (b == 0) {  // one CTA writes the routing outputs and the w2 kernel's tables
+      if (warp == 1) publish_tables(S.tb, P);
+      if (P.layer_mode && warp == 2)
+        for (int i = lane; i < T * P.k; i += 32) {
+          P.topk_ids[i] = S.rt.sel_ids[i];
+          P.topk_w[i] = S.rt.sel_w[i];
+        }
+      if (P.layer_mode && warp == 3) write_permutation(S.rt, P, S.tb.nh);
+    }
+    prep_x();
+  }
+  if (q == 1) {
+    // group 0's tables, before this group's first routed position
+    uint32_t i = 0;
+    while (*reinterpret_cast<volatile int*>(&S.ready) == 0 && ++i < kBarTries) __nanosleep(32);
+    if (i >= kBarTries) {
+      ok = false;
+      if (lane == 0) atomicOr(P.status, kStatusTimeout);
+    }
+    __threadfence_block();
+  }
+  const Chunk ch = w13_chunk(P, S.tb.nh, b, G);
+  const int npos = ch.size();
+
+  // ---- item loop: group q takes ring positions nsp + q, nsp + q + 2, ...
+  for (int pos = nsp + q; pos < npos && ok; pos += 2) ok = run_item(ch, npos, pos, true, false);
+  // No copy may still be landing in this CTA's shared memory (possible only
+  // after a timeout).
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int s = 0; s < kStages13; ++s)
+      if (S.lastfill[s] >= 0) mbar_wait_bounded(&S.full[s], uint32_t(S.lastfill[s] / kStages13) & 1u, kBarTries);
+}
+
+// ---------------------------------------------------------------- w2 kernel
+
+struct W2Smem {
+  uint64_t full[kMaxStages2];
+  int redcnt[kMaxStages2];
+  int lastfill[kMaxStages2];
+  float sh_scale[kShRows];  // shared-expert row scales of this CTA's output rows
+  Tables tb;
+};
+constexpr size_t kHead2 = (sizeof(W2Smem) + 127) / 128 * 128;
+constexpr size_t kRed2 = size_t(16) * 32 * 16;  // float4 per lane and warp
+
+// Ring position p of CTA b: output block rb = b w2_per + p / nl, expert slot
+// l = p % nl (the shared expert first when there is one, then the routed list).
+struct Item2 {
+  int rb, l, li;  // li < 0: shared expert
+};
+__device__ __forceinline__ Item2 w2_item(const DecParams& P, int nl, int b, int p) {
+  Item2 m;
+  m.rb = b * P.w2_per + p / nl;
+  m.l = p % nl;
+  m.li = P.Is > 0 ? m.l - 1 : m.l;
+  return m;
+}
+
+// Offset of the token rows of intermediates in a stage.
+__device__ __forceinline__ int w2_hoff(const DecParams& P) {
+  return max(16 * P.Is, 16 * (P.I / 2) + 16 * (P.I / 32));
+}
+
+// Weight rows [rb * 16, +16) of the item's expert: adds their bytes to the
+// stage's barrier without arriving (lane 0).
+__device__ __forceinline__ void fill2_weights(const DecParams& P, W2Smem& S, char* dst, int s, const Item2& m) {
+  if (m.li < 0) {
+    mbar_expect_tx(&S.full[s], uint32_t(16 * P.Is));
+    bulk_g2s(dst, reinterpret_cast<const char*>(P.sh2) + size_t(m.rb) * 16 * P.Is, uint32_t(16 * P.Is), &S.full[s]);
+  } else {
+    const size_t r0 = size_t(S.tb.hit[m.li]) * P.H + size_t(m.rb) * 16;
+    mbar_expect_tx(&S.full[s], uint32_t(16 * (P.I / 2) + 16 * (P.I / 32)));
+    bulk_g2s(dst, P.w2_codes + r0 * (P.I / 2), uint32_t(16 * (P.I / 2)), &S.full[s]);
+    bulk_g2s(dst + 16 * (P.I / 2), P.w2_scales + r0 * (P.I / 32), uint32_t(16 * (P.I / 32)), &S.full[s]);
+  }
+}
+
+// The intermediates of the expert's tokens (token t in slot t), then the
+// stage's one arrival (whole warp). Only after the w13 grid is complete.
+__device__ __forceinline__ void fill2_h(const DecParams& P, W2Smem& S, char* dst, int s, const Item2& m) {
+  const int lane = threadIdx.x & 31;
+  const bool sh = m.li < 0;
+  const int K = sh ? P.Is : P.I;
+  const uint32_t mask = sh ? (1u << P.T) - 1u : S.tb.mask[m.li];
+  if (lane == 0) mbar_arrive_expect_tx(&S.full[s], uint32_t(__popc(mask)) * uint32_t(K * 2));
+  __syncwarp();
+  if (lane < P.T && ((mask >> lane) & 1u)) {
+    const __half* src = sh ? P.hs + size_t(lane) * P.Is : P.dh + (size_t(m.li) * P.T + lane) * P.I;
+    bulk_g2s(dst + w2_hoff(P) + lane * K * 2, src, uint32_t(K * 2), &S.full[s]);
+  }
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
+  extern __shared__ __align__(128) char smem[];
+  W2Smem& S = *reinterpret_cast<W2Smem*>(smem);
+  char* stages = smem + kHead2;
+  float4* red = reinterpret_cast<float4*>(stages + size_t(P.nstages) * P.stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int T = P.T, NS = P.nstages;
+  const int b = int(blockIdx.x);
+  const int nrb_mine = max(0, min(P.w2_per, P.H / 16 - b * P.w2_per));
+  const bool has_sh = P.Is > 0;
+
+  // row scales first: a global load waits behind the SM's copies in flight
+  if (has_sh)
+    for (int i = threadIdx.x; i < 16 * nrb_mine && i < kShRows; i += blockDim.x)
+      S.sh_scale[i] = __ldg(P.sh2_scale + 16 * b * P.w2_per + i);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&S.full[s], 1);
+      S.redcnt[s] = 0;
+      S.lastfill[s] = -1;
+    }
+    fence_mbar_init();
+    // Position 0 is the shared expert of the first block: its weight rows do
+    // not depend on the previous grids.
+    if (has_sh && nrb_mine > 0) fill2_weights(P, S, stages, 0, Item2{b * P.w2_per, 0, -1});
+  }
+  __syncthreads();
+  pdl_wait();
+  read_tables(S.tb, P);
+  __syncthreads();
+  const int nl = S.tb.nh + (has_sh ? 1 : 0);
+  const int n_items = nrb_mine * nl;
+  if (warp == 0)
+    for (int p = 0; p < NS && p < n_items; ++p) {
+      const Item2 m = w2_item(P, nl, b, p);
+      if (lane == 0) {
+        S.lastfill[p] = p;
+        if (!(p == 0 && has_sh)) fill2_weights(P, S, stages + size_t(p) * P.stage_bytes, p, m);
+      }
+      __syncwarp();
+      fill2_h(P, S, stages + size_t(p) * P.stage_bytes, p, m);
+    }
+  // Position 0's shared weights were armed before the wait even if it turns
+  // out there is nothing to do; give that copy its arrival so it can land.
+  if (warp == 0 && n_items == 0 && has_sh && nrb_mine > 0 && lane == 0) {
+    S.lastfill[0] = 0;
+    mbar_arrive(&S.full[0]);
+  }
+
+  // Two groups of eight warps take alternate expert slots of each output
+  // block; warp i of a group owns K blocks i, i + 8. Every warp keeps its
+  // partial sums over the block's experts in registers; at the end of the
+  // block all sixteen are summed in warp order.
+  const int q = warp >> 3, wi = warp & 7;
+  bool ok = true;
+  for (int r = 0; r < nrb_mine; ++r) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int l = q; l < nl; l += 2) {
+      const int pos = r * nl + l;
+      const Item2 m = w2_item(P, nl, b, pos);
+      const int s = pos % NS;
+      // A timed-out warp keeps going (without reading the stage) so that every
+      // warp reaches the block-end barriers.
+      ok = ok && __all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / NS) & 1u, P));
+      if (!ok) continue;
+      const char* st = stages + size_t(s) * P.stage_bytes;
+      const bool sh = m.li < 0;
+      const int K = sh ? P.Is : P.I;
+      const int nkb = K / 128;
+      // B: the intermediates of token g (zero for tokens not routed here)
+      const uint32_t mask = sh ? (1u << T) - 1u : S.tb.mask[m.li];
+      const bool has_tok = g < T && ((mask >> g) & 1u);
+      uint32_t Bf[2][16];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int kb = wi + 8 * j;
+        if (has_tok && kb < nkb) {
+          const uint4* p4 = reinterpret_cast<const uint4*>(st + w2_hoff(P) + g * K * 2 + kb * 256 + 64 * t);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const uint4 v = p4[p];
+            Bf[j][4 * p] = v.x;
+            Bf[j][4 * p + 1] = v.y;
+            Bf[j][4 * p + 2] = v.z;
+            Bf[j][4 * p + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) Bf[j][i] = 0u;
+        }
+      }
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+      if (sh) {
+        tile_s8<2, 8>(st + g * P.Is, st + (g + 8) * P.Is, true, 0, nkb, wi, Bf, a0, a1);
+        const int rl = (m.rb - b * P.w2_per) * 16 + g;  // row within this CTA's output rows
+        const float its = 1.0f / P.tau_s;
+        const float sa = (rl < kShRows ? S.sh_scale[rl] : __ldg(P.sh2_scale + m.rb * 16 + g)) * its;
+        const float sb = (rl + 8 < kShRows ? S.sh_scale[rl + 8] : __ldg(P.sh2_scale + m.rb * 16 + g + 8)) * its;
+        acc.x += (a0[0] + a1[0]) * sa;
+        acc.y += (a0[1] + a1[1]) * sa;
+        acc.z += (a0[2] + a1[2]) * sb;
+        acc.w += (a0[3] + a1[3]) * sb;
+      } else {
+        const int rs = P.I / 2, Gs = P.I / 32;
+        const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + 16 * rs);
+        float fa, fb;
+        tile_mx<2, 8>(st + g * rs, st + (g + 8) * rs, sc + g * Gs, sc + (g + 8) * Gs, wi, nkb, Bf, a0, a1, fa, fb);
+        fa *= 1.0f / P.tau_r;
+        fb *= 1.0f / P.tau_r;
+        acc.x += (a0[0] + a1[0]) * fa;
+        acc.y += (a0[1] + a1[1]) * fa;
+        acc.z += (a0[2] + a1[2]) * fb;
+        acc.w += (a0[3] + a1[3]) * fb;
+      }
+      // the last warp of the group to finish with the stage refills it
+      __syncwarp();
+      int old = 0;
+      if (lane == 0) old = atomicAdd(&S.redcnt[s], 1);
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (old == 7) {
+        if (lane == 0) S.redcnt[s] = 0;
+        __syncwarp();
+        const int np = pos + NS;
+        if (np < n_items) {
+          const Item2 mn = w2_item(P, nl, b, np);
+          if (lane == 0) {
+            S.lastfill[s] = np;
+            fill2_weights(P, S, stages + size_t(s) * P.stage_bytes, s, mn);
+          }
+          __syncwarp();
+          fill2_h(P, S, stages + size_t(s) * P.stage_bytes, s, mn);
+        }
+      }
+    }
+    // block done: sum the 16 warps' partials in warp order, write bf16
+    red[warp * 32 + lane] = acc;
+    __syncthreads();
+    if (warp == 0) {
+      float4 d = red[lane];
+      for (int w = 1; w < 16; ++w) {
+        const float4 v = red[w * 32 + lane];
+        d.x += v.x;
+        d.y += v.y;
+        d.z += v.z;
+        d.w += v.w;
+      }
+      const float v[4] = {d.x, d.y, d.z, d.w};
+      const int rb = b * P.w2_per + r;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tok = 2 * t + (i & 1);
+        if (tok < T) P.out[size_t(tok) * P.H + rb * 16 + g + 8 * (i >> 1)] = __float2bfloat16_rn(v[i]);
+      }
+    }
+    __syncthreads();
+  }
+  // No copy may still be landing in this CTA's shared memory.
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int s = 0; s < NS; ++s)
+      if (S.lastfill[s] >= 0) mbar_wait_bounded(&S.full[s], uint32_t(S.lastfill[s] / NS) & 1u, kBarTries);
+}
+
+// ---------------------------------------------------------------- host side
+
+// 2^e for the largest e <= 14 with bound * 2^e below the f16 maximum.
+float h_scale(float bound) {
+  int e = 0;
+  while (e < 14 && bound * std::ldexp(1.0f, e + 1) < 65504.0f) ++e;
+  return std::ldexp(1.0f, e);
+}
+
+struct Plan {
+  int stage13 = 0, stage2 = 0, nst2 = 0;
+  size_t smem13 = 0, smem2 = 0;
+  bool ok = false;
+};
+
+Plan make_plan(const v4moe_config& c, int T) {
+  Plan p;
+  if (T < 1 || T > kDecodeMaxTokens || T * c.top_k > kMaxHit) return p;
+  const int H = c.hidden, I = c.inter, Is = c.shared_inter;
+  if (H > kNJ * 8 * 128 || I > 2 * 8 * 128 || Is > 2 * 8 * 128) return p;
+  int s13 = 16 * (H / 2) + 16 * (H / 32);
+  if (Is > 0) s13 = std::max(s13, 8 * H);
+  p.stage13 = (s13 + 127) / 128 * 128;
+  const size_t route_stage = (size_t(T) * c.n_experts + c.n_experts) * 4;  // scores + bias
+  p.smem13 = kHead13 + size_t(kStages13) * p.stage13 + kPart13 + (route_stage + 127) / 128 * 128;
+  const int hoff = std::max(16 * Is, 16 * (I / 2) + 16 * (I / 32));
+  const int s2 = hoff + T * std::max(I, Is) * 2;
+  p.stage2 = (s2 + 127) / 128 * 128;
+  const size_t room = 227 * 1024 - kHead2 - kRed2;
+  p.nst2 = int(std::min<size_t>(kMaxStages2, room / p.stage2));
+  p.smem2 = kHead2 + size_t(p.nst2) * p.stage2 + kRed2;
+  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 &&
+         size_t(T) * H * 2 <= 227 * 1024;
+  return p;
+}
+
+}  // namespace
+
+DecodeBuffers dec_buffers(const v4moe_config& c, int64_t T) {
+  DecodeBuffers b;
+  if (T < 1 || T > kDecodeMaxTokens) return b;
+  b.ctl = size_t(cWords) * 4;
+  b.dh = size_t(kMaxHit) * T * c.inter * 2;
+  b.hs = size_t(T) * std::max(c.shared_inter, 0) * 2;
+  return b;
+}
+
+bool dec_supported(const v4moe_config& c, int T) { return make_plan(c, T).ok; }
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
+  const v4moe_config& c = a.c;
+  const Plan p = make_plan(c, a.T);
+  if (!p.ok) return cudaErrorInvalidValue;
+  const int sms = device_sms();
+  DecParams P;
+  P.T = a.T;
+  P.H = c.hidden;
+  P.I = c.inter;
+  P.Is = c.shared_inter;
+  P.E = c.n_experts;
+  P.k = c.top_k;
+  P.vocab = c.vocab;
+  P.limit = c.swiglu_limit;
+  P.routed_scale = c.routed_scale;
+  // |h| <= L * L * |routed_scale| (routed weights sum to routed_scale) and
+  // L * L (shared): the largest power of two that keeps h * tau below the f16
+  // maximum gives small intermediates that many more binades
+  const float L = c.swiglu_limit;
+  P.tau_r = h_scale(L * L * std::max(1.0f, std::fabs(c.routed_scale)));
+  P.tau_s = h_scale(L * L);
+  P.layer_mode = a.layer_mode;
+  P.stage_bytes = 0;
+  P.nstages = 0;
+  P.w2_per = 1;
+  P.x = a.x;
+  P.gate = a.gate;
+  P.bias = a.bias;
+  P.token_ids = a.token_ids;
+  P.tid2eid = a.tid2eid;
+  P.topk_ids = a.topk_ids;
+  P.topk_w = a.topk_w;
+  P.counts = a.counts;
+  P.offsets = a.offsets;
+  P.sorted_slot = a.sorted_slot;
+  P.slot_pos = a.slot_pos;
+  P.scores = a.scores;
+  P.w13_codes = a.w.w13_codes;
+  P.w13_scales = a.w.w13_scales;
+  P.w2_codes = a.w.w2_codes;
+  P.w2_scales = a.w.w2_scales;
+  P.sh13 = a.w.sh_w13;
+  P.sh13_scale = a.w.sh_w13_scale;
+  P.sh2 = a.w.sh_w2;
+  P.sh2_scale = a.w.sh_w2_scale;
+  P.dh = a.dh;
+  P.hs = a.hs;
+  P.ctl = a.ctl;
+  P.status = a.status;
+  P.out = a.out;
+
+  const int nrb = c.hidden / 16;
+  P.w2_per = (nrb + sms - 1) / sms;
+  const int grid2 = (nrb + P.w2_per - 1) / P.w2_per;
+  cudaError_t e = cudaSuccess;
+  if (a.layer_mode) {
+    const size_t route_smem = size_t(a.T) * c.hidden * 2;
+    set_smem(k_dec_route, route_smem);
+    e = launch_kernel("dec_route", k_dec_route, dim3((c.n_experts + kRouteWarps - 1) / kRouteWarps),
+                      dim3(kRouteWarps * 32), route_smem, st, false, P);
+    if (e != cudaSuccess) return e;
+  }
+  // Without a routing kernel in front, the w13 kernel must not overlap the
+  // previous call's w2 kernel (it rewrites the intermediates that one reads).
+  P.stage_bytes = p.stage13;
+  set_smem(k_dec_w13, p.smem13);
+  e = launch_kernel("dec_w13", k_dec_w13, dim3(sms), dim3(kThreads), p.smem13, st, a.layer_mode != 0, P);
+  if (e != cudaSuccess) return e;
+  P.stage_bytes = p.stage2;
+  P.nstages = p.nst2;
+  set_smem(k_dec_w2, p.smem2);
+  return launch_kernel("dec_w2", k_dec_w2, dim3(grid2), dim3(kThreads), p.smem2, st, true, P);
+}
+
+}  // namespace v4moe

@@ -7,7 +7,7 @@
 // "config.json" experts_w4a16): for every routed expert e and its tokens
 // (slots in expert order),
 //   w13: [g; u] = W13_e[{j, I+j}] x (fp32), h = silu(min(g, L)) * clamp(u, -L, L);
-//   w2:  y_slot = W2_e h (fp32); the combine kernel forms the output.
+//   w2:  y_slot = bf16(W2_e h); the combine forms the output.
 //
 // Exact activations: a bf16 value has 8 significant bits. Per block of 32
 // values with largest magnitude a, the scale 2^s (s the smallest exponent with
@@ -94,7 +94,7 @@ struct MxParams {
   uint8_t* h_lo;
   uint8_t* hs_hi;           // w13 out: [S, I/32] E8M0
   uint8_t* hs_lo;
-  float* y_slot;            // w2 out: [S, H]
+  __nv_bfloat16* y_slot;    // w2 out: [S, H] bf16
   uint32_t* status;
 };
 
@@ -575,7 +575,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int col = c0 + i;
-            if (col < g.n) P.y_slot[size_t(g.brow0 + col) * P.H + m] = __uint_as_float(rv[i]);
+            if (col < g.n) P.y_slot[size_t(g.brow0 + col) * P.H + m] = __float2bfloat16_rn(__uint_as_float(rv[i]));
           }
         }
       }
@@ -922,15 +922,19 @@ __global__ void __launch_bounds__(kXThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.acc_empty);
         if (valid) {
-          float4* dy = reinterpret_cast<float4*>(P.y_slot + slot * P.H + t.row0 + 64 * sub);
+          uint4* dy = reinterpret_cast<uint4*>(P.y_slot + slot * P.H + t.row0 + 64 * sub);
+          auto pk = [](uint32_t a, uint32_t b) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(a), __uint_as_float(b));
+            return *reinterpret_cast<const uint32_t*>(&v);
+          };
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dy[i] = make_float4(__uint_as_float(ya[4 * i]), __uint_as_float(ya[4 * i + 1]),
-                                __uint_as_float(ya[4 * i + 2]), __uint_as_float(ya[4 * i + 3]));
+          for (int i = 0; i < 4; ++i)
+            dy[i] = make_uint4(pk(ya[8 * i], ya[8 * i + 1]), pk(ya[8 * i + 2], ya[8 * i + 3]),
+                               pk(ya[8 * i + 4], ya[8 * i + 5]), pk(ya[8 * i + 6], ya[8 * i + 7]));
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dy[8 + i] = make_float4(__uint_as_float(yb[4 * i]), __uint_as_float(yb[4 * i + 1]),
-                                    __uint_as_float(yb[4 * i + 2]), __uint_as_float(yb[4 * i + 3]));
+          for (int i = 0; i < 4; ++i)
+            dy[4 + i] = make_uint4(pk(yb[8 * i], yb[8 * i + 1]), pk(yb[8 * i + 2], yb[8 * i + 3]),
+                                   pk(yb[8 * i + 4], yb[8 * i + 5]), pk(yb[8 * i + 6], yb[8 * i + 7]));
         }
       }
     }

@@ -87,7 +87,7 @@ struct TcParams {
   const float* sh_scale;            // shared expert fp32 row scales
   __half* h;                        // w13 out: [S, I]
   __half* hs;                       // w13 out: [T, Is]
-  float* y_slot;                    // w2 out: [S, H]
+  __nv_bfloat16* y_slot;            // w2 out: [S, H] bf16
   float* ys;                        // w2 out: [T, H]
   uint32_t* status;
 };
@@ -443,12 +443,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           named_bar_sync(1, 128);
         } else {
-          float* yout = g.shared ? P.ys : P.y_slot;
           const int m = t.row0 + row;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int col = c0 + i;
-            if (col < g.n) yout[size_t(g.brow0 + col) * P.H + m] = __uint_as_float(rv[i]) * rowf;
+            if (col < g.n) {
+              const float v = __uint_as_float(rv[i]) * rowf;
+              if (g.shared)
+                P.ys[size_t(g.brow0 + col) * P.H + m] = v;
+              else
+                P.y_slot[size_t(g.brow0 + col) * P.H + m] = __float2bfloat16_rn(v);
+            }
           }
         }
       }

@@ -7,7 +7,7 @@
 // output channel):
 //   w13: hs[t, c] = silu(min(s_g[c] g, L)) * clamp(s_u[c] u, -L, L),
 //        g = q13[c] . x_t, u = q13[Is + c] . x_t                     (f16 out)
-//   w2:  out[t, m] = bf16( sum_j w[t, j] y_slot[slot(t, j), m] + s2[m] (q2[m] . hs_t) )
+//   w2:  out[t, m] = bf16( sum_j w[t, j] y_slot[slot(t, j), m] + s2[m] (q2[m] . hs_t) )  (y_slot bf16)
 // with the routed expert outputs y_slot of the same call, summed in slot order
 // j = 0 .. k-1 and then the shared term, so the result does not depend on
 // timing.
@@ -88,7 +88,7 @@ struct ShParams {
   const int32_t* topk_ids;
   const float* topk_w;
   const int32_t* slot_pos;
-  const float* y_slot;   // [T k, H] routed outputs in slot order
+  const __nv_bfloat16* y_slot;  // [T k, H] routed outputs in slot order (bf16)
   __nv_bfloat16* out;    // [T, H]; linear mode: [T, G N]
   // linear mode: G groups of N output channels over K inputs each (group g
   // reads x columns g K .. and weight rows g N ..); bn weight rows per tile
@@ -144,21 +144,21 @@ __device__ __forceinline__ void combine_round(const ShParams& P, const float (&w
     const int tl = 4 * g + sl;  // token within the warp's 32
     float w[NJ];
     int p[NJ];
-    float4 y[NJ];
+    uint2 y[NJ];
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       w[j] = __shfl_sync(0xffffffffu, wj[j], tl);
       p[j] = __shfl_sync(0xffffffffu, pj[j], tl);
-      y[j] = __ldg(reinterpret_cast<const float4*>(P.y_slot + size_t(max(p[j], 0)) * P.H + m0 + c4));
+      y[j] = __ldg(reinterpret_cast<const uint2*>(P.y_slot + size_t(max(p[j], 0)) * P.H + m0 + c4));
     }
     float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       if (p[j] >= 0) {
-        a.x = fmaf(w[j], y[j].x, a.x);
-        a.y = fmaf(w[j], y[j].y, a.y);
-        a.z = fmaf(w[j], y[j].z, a.z);
-        a.w = fmaf(w[j], y[j].w, a.w);
+        a.x = fmaf(w[j], __uint_as_float(y[j].x << 16), a.x);
+        a.y = fmaf(w[j], __uint_as_float(y[j].x & 0xFFFF0000u), a.y);
+        a.z = fmaf(w[j], __uint_as_float(y[j].y << 16), a.z);
+        a.w = fmaf(w[j], __uint_as_float(y[j].y & 0xFFFF0000u), a.w);
       }
     }
     const int t2 = tq + tl;

@@ -174,7 +174,7 @@ ForwardArgs forward_args(const v4moe_config* cfg, int32_t T, const void* x, cons
   a.out = static_cast<__nv_bfloat16*>(out);
   a.status = at<uint32_t>(ws, L.status);
   a.h = at<__nv_bfloat16>(ws, L.h);
-  a.y_slot = at<float>(ws, L.y_slot);
+  a.y_slot = at<__nv_bfloat16>(ws, L.y_slot);
   a.hs = at<__nv_bfloat16>(ws, L.hs);
   a.ys = at<float>(ws, L.ys);
   return a;
@@ -195,7 +195,7 @@ DecodeArgs decode_args(const v4moe_config* cfg, int32_t T, const void* x, const 
   d.scores = at<float>(ws, L.scores);
   d.ctl = at<uint32_t>(ws, L.d_ctl);
   d.dh = at<__half>(ws, L.d_dh);
-  d.part = at<float>(ws, L.d_part);
+  d.hs = at<__half>(ws, L.d_hs);
   return d;
 }
 
@@ -221,7 +221,7 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x, const i
   if (T == 0) return V4MOE_OK;
   const WsLayout L = ws_layout(*cfg, T);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dec_supported(*cfg, T, *weights)) {
+  if (dec_supported(*cfg, T)) {
     DecodeArgs d = decode_args(cfg, T, x, weights, out, ws);
     d.layer_mode = 0;
     d.topk_ids = const_cast<int32_t*>(topk_ids);
@@ -252,7 +252,7 @@ int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const voi
   if (int32_t r = check_device()) return r;
   // an empty batch still reports empty counts and offsets
   if (T == 0) return v4moe_permute(cfg, 0, topk_ids, counts, offsets, sorted_slot, slot_pos, ws, ws_bytes, stream);
-  if (dec_supported(*cfg, T, *weights)) {
+  if (dec_supported(*cfg, T)) {
     DecodeArgs d = decode_args(cfg, T, x, weights, out, ws);
     d.layer_mode = 1;
     d.gate = static_cast<const __nv_bfloat16*>(gate);

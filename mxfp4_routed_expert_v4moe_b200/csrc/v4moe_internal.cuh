@@ -42,11 +42,10 @@ int route_ksplit(const v4moe_config& c, int64_t T);
 constexpr int kShMinTokens = 512;
 size_t sh_extra_bytes(const v4moe_config& c, int64_t T);
 
-// Buffers of the decode path (all zero bytes when T is above its limit): ctl
-// holds counters that are zero at rest, dh the intermediates, part the w2
-// partial sums per expert.
+// Buffers of the decode path (all zero bytes when T is above its limit). ctl
+// holds the routing tables.
 struct DecodeBuffers {
-  size_t ctl = 0, dh = 0, part = 0;
+  size_t ctl = 0, dh = 0, hs = 0;
 };
 DecodeBuffers dec_buffers(const v4moe_config& c, int64_t T);
 
@@ -57,14 +56,14 @@ struct WsLayout {
   size_t chunk_counts = 0;  // [nchunks, E] int32
   size_t chunk_base = 0;    // [nchunks, E] int32
   size_t h = 0;             // [T*k, I] bf16 routed intermediates (sorted order)
-  size_t y_slot = 0;        // [T*k, H] fp32 routed expert outputs (sorted order)
+  size_t y_slot = 0;        // [T*k, H] bf16 routed expert outputs (sorted order)
   size_t hs = 0;            // [T, I_s] bf16 shared intermediates
   size_t ys = 0;            // [T, H] fp32 shared expert outputs
   size_t xlog = 0;          // [T, H] f16 activations in the decode layout
   size_t sigma = 0;         // [T] int32 per-token power-of-two exponents
   size_t tc = 0;            // tensor-core path: activations in slot order + tile lists
   size_t sh16 = 0;          // shared expert weights widened to f16 (large batches)
-  size_t d_ctl = 0, d_dh = 0, d_part = 0;  // decode path
+  size_t d_ctl = 0, d_dh = 0, d_hs = 0;  // decode path
   size_t total = 0;
   int nchunks = 0;
 };
@@ -85,7 +84,7 @@ inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
   L.chunk_counts = take(size_t(L.nchunks) * c.n_experts * 4);
   L.chunk_base = take(size_t(L.nchunks) * c.n_experts * 4);
   L.h = take(size_t(S) * c.inter * 2);
-  L.y_slot = take(size_t(S) * c.hidden * 4);
+  L.y_slot = take(size_t(S) * c.hidden * 2);
   L.hs = take(size_t(T) * (c.shared_inter > 0 ? c.shared_inter : 0) * 2);
   L.ys = take(size_t(T) * c.hidden * 4);
   L.xlog = take(size_t(T) * c.hidden * 2);
@@ -95,7 +94,7 @@ inline WsLayout ws_layout(const v4moe_config& c, int64_t T) {
   const DecodeBuffers d = dec_buffers(c, T);
   L.d_ctl = take(d.ctl);
   L.d_dh = take(d.dh);
-  L.d_part = take(d.part);
+  L.d_hs = take(d.hs);
   L.total = off;
   return L;
 }
@@ -128,7 +127,7 @@ struct ForwardArgs {
   // workspace pieces
   uint32_t* status;
   __nv_bfloat16* h;
-  float* y_slot;
+  __nv_bfloat16* y_slot;  // routed expert outputs, bf16 (16-bit activations)
   __nv_bfloat16* hs;
   float* ys;
 };
@@ -179,8 +178,9 @@ cudaError_t launch_linear_w8a16(int T, int G, int N, int K, const __nv_bfloat16*
 cudaError_t launch_forward_tc(const ForwardArgs& a, __half* x16, int* sigma, char* extra, char* sh16,
                               cudaStream_t st);
 
-// Decode path: the whole layer (routing included in layer mode) in one
-// persistent kernel, for at most kDecodeMaxTokens tokens.
+// Decode path: the whole layer (routing included in layer mode) as three
+// kernels chained by programmatic dependent launch, for at most
+// kDecodeMaxTokens tokens.
 constexpr int kDecodeMaxTokens = 8;
 struct DecodeArgs {
   v4moe_config c;
@@ -203,9 +203,9 @@ struct DecodeArgs {
   uint32_t* status;
   uint32_t* ctl;
   __half* dh;
-  float* part;
+  __half* hs;
 };
-bool dec_supported(const v4moe_config& c, int T, const v4moe_weights& w);
+bool dec_supported(const v4moe_config& c, int T);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- device helpers

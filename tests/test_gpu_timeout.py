@@ -1,9 +1,9 @@
-"""Failure detection on the GPU without a fault: every device-side wait of the
-decode kernel is bounded. Word 1 of the workspace's status block, when
-non-zero, makes the router's wait expect one more CTA than the grid has and
-caps it at that many polls; the wait then gives up, the kernel sets the
-timeout bit of the status word, waits for its own copies and returns, and
-the context stays usable. Clearing the status block disarms it."""
+"""Failure detection on the GPU without a fault: device-side waits are
+bounded. Word 1 of the workspace's status block, when non-zero, makes the
+decode expert kernel wait on a barrier that nothing arrives at, capped at that
+many polls; the wait gives up, the kernel sets the timeout bit of the status
+word and returns, and the context stays usable. Clearing the status block
+disarms it."""
 import numpy as np
 import pytest
 
@@ -25,7 +25,7 @@ def test_router_wait_gives_up_then_the_next_call_is_exact():
     x, bias, _, _ = upload_activations(li)
     ws = layer.workspace(wl.T)
     assert V.v4moe_clear_device_status(ws) == V.V4MOE_OK
-    ws[:256].view(torch.int32)[1] = 2000   # arm: the router wait can never be met
+    ws[:256].view(torch.int32)[1] = 2000   # arm: a wait that can never be met
     layer(x, bias)
     assert V.v4moe_read_device_status(ws) == V.V4MOE_ERR_TIMEOUT
     # the context is intact and the counters were reset: clear and run again
