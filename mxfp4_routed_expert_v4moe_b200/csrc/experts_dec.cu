@@ -46,14 +46,21 @@
 // binades; the down projection divides it out.
 //
 // Operands are exact: E2M1 pairs via cvt.rn.f16x2.e2m1x2, int8 via a
-// magic-number conversion; the E8M0 group scale multiplies the f16 operand as
-// a power of two relative to the largest exponent among the warp's groups of
-// that row, and the rest is applied in fp32. Activations are f16, scaled per
-// token by a power of two that puts the row maximum in [2^14, 2^15).
+// magic-number conversion. Each 32-wide scale group is its own pair of MMAs
+// started from zero, and its E8M0 scale multiplies that result in fp32.
+// Activations are f16, scaled per token by a power of two that puts the row
+// maximum in [2^14, 2^15).
+//
+// Weight slabs arrive by TMA as swizzled boxes (a few copies per slab, and
+// the eight rows of every fragment load in different banks). A stage's
+// consecutive ring positions go to different consumers, so besides its
+// mbarrier each stage carries a tag naming the position whose copies were
+// issued; a consumer waits for the tag before it tests the barrier's parity.
 //
 // No CTA waits on another CTA: data crosses kernels only at the programmatic
 // launch boundaries (griddepcontrol.wait), which also order memory. Every
-// mbarrier wait is bounded and flags the status word.
+// wait is bounded and flags the status word.
+#include <cuda.h>
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -121,6 +128,14 @@ struct DecParams {
   __nv_bfloat16* out;
 };
 
+// Tensor maps of a slab kernel's weights (u8 views, built on the host):
+// codes {128, rows, K / 256 chunks} with box {128, 8 or 16, K / 256}, scales
+// {K / 32, rows} with box {K / 32, 8 or 16}, shared-expert int8 rows {128,
+// rows, K / 128} with box {128, 4 or 16, K / 128}.
+struct DecMaps {
+  CUtensorMap codes, scales, shared;
+};
+
 // Routing tables as the slab kernels keep them in shared memory.
 struct Tables {
   int nh;
@@ -138,6 +153,23 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const D
   if (mbar_wait_bounded(bar, parity, kBarTries)) return true;
   atomicOr(P.status, kStatusTimeout);
   return false;
+}
+
+// Waits until ring stage `bar` / `tag` holds position pos of a ring of ns
+// stages. Consecutive positions of a stage (pos - ns, pos) go to different
+// consumers, so a consumer can reach pos while the stage still holds pos - ns;
+// the barrier's parity alone would then take the older phase's completion for
+// this one. The tag names the last position whose copies were issued: it is
+// written after pos - ns was consumed and before pos's copies, so once it
+// reads pos the barrier's current phase is pos's.
+__device__ __forceinline__ bool wait_stage(uint64_t* bar, const int* tag, int pos, int ns, const DecParams& P) {
+  uint32_t i = 0;
+  while (*reinterpret_cast<const volatile int*>(tag) != pos && ++i < kBarTries) __nanosleep(20);
+  if (i >= kBarTries) {
+    atomicOr(P.status, kStatusTimeout);
+    return false;
+  }
+  return wait_bar(bar, uint32_t(pos / ns) & 1u, P);
 }
 
 // 14 - floor(log2 m) for the largest bf16 magnitude bits m of a row (0 for an
@@ -166,90 +198,122 @@ __device__ __forceinline__ void read_tables(Tables& tb, const DecParams& P) {
 
 // ---------------------------------------------------------------- slab products
 
-// MXFP4 m16 tile: rows g and g + 8 of the tile at ra / rb (codes of 128-wide
-// K block kb at kb * 64), their E8M0 scale rows at sa / sb. The warp's K
-// blocks kb = wi + KS j (j < NJ, kb < nkb) multiply B[j]. Even and odd MMA
-// steps go to separate accumulators; fa / fb get the fp32 factors of the two
-// rows.
-template <int NJ, int KS>
-__device__ __forceinline__ void tile_mx(const char* ra, const char* rb, const uint8_t* sa, const uint8_t* sb, int wi,
-                                        int nkb, const uint32_t (&B)[NJ][16], float (&ae)[4], float (&ao)[4],
-                                        float& fa, float& fb) {
-  const int t = threadIdx.x & 3;
-  int xa = 0, xb = 0;
-#pragma unroll
-  for (int j = 0; j < NJ; ++j) {
-    const int kb = wi + KS * j;
-    if (kb < nkb) {
-      xa = max(xa, int(sa[4 * kb + t]));
-      xb = max(xb, int(sb[4 * kb + t]));
-    }
-  }
-  xa = max(xa, __shfl_xor_sync(0xffffffffu, xa, 1));
-  xa = max(xa, __shfl_xor_sync(0xffffffffu, xa, 2));
-  xb = max(xb, __shfl_xor_sync(0xffffffffu, xb, 1));
-  xb = max(xb, __shfl_xor_sync(0xffffffffu, xb, 2));
-#pragma unroll
-  for (int j = 0; j < NJ; ++j) {
-    const int kb = wi + KS * j;
-    if (kb < nkb) {
-      const uint4 qa = *reinterpret_cast<const uint4*>(ra + kb * 64 + 16 * t);
-      const uint4 qb = *reinterpret_cast<const uint4*>(rb + kb * 64 + 16 * t);
-      const uint32_t fsa = f16_pow2_bits(int(sa[4 * kb + t]) - xa + 13) * 0x10001u;
-      const uint32_t fsb = f16_pow2_bits(int(sb[4 * kb + t]) - xb + 13) * 0x10001u;
-      const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w};
-      const uint32_t wb[4] = {qb.x, qb.y, qb.z, qb.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        uint32_t ca[4], cb[4];
-        e2m1x8_to_f16x2(wa[u], ca);
-        e2m1x8_to_f16x2(wb[u], cb);
-        const uint32_t A0[4] = {hmul2_u32(ca[0], fsa), hmul2_u32(cb[0], fsb), hmul2_u32(ca[1], fsa),
-                                hmul2_u32(cb[1], fsb)};
-        const uint32_t A1[4] = {hmul2_u32(ca[2], fsa), hmul2_u32(cb[2], fsb), hmul2_u32(ca[3], fsa),
-                                hmul2_u32(cb[3], fsb)};
-        mma_16816_f16(ae, A0, B[j][4 * u], B[j][4 * u + 1]);
-        mma_16816_f16(ao, A1, B[j][4 * u + 2], B[j][4 * u + 3]);
-      }
-    }
-  }
-  fa = pow2f(xa - 127 - 13);
-  fb = pow2f(xb - 127 - 13);
+// Slab layout in a stage. Weight rows arrive by TMA as boxes {128 bytes,
+// rows, chunks}: chunk c (bytes 128 c .. 128 c + 127) of every row of the box,
+// then chunk c + 1, ..., so row r's chunk c is line c * rows + r of the box.
+// The 128-byte swizzle permutes the eight 16-byte units of each line by the
+// line index mod 8; the eight rows a fragment load touches are eight
+// consecutive lines, so their units fall in eight different bank groups. Row
+// scales arrive as boxes {S bytes, rows} (S = K / 32) with the swizzle of span
+// S (none at 16 bytes). Every box starts at a multiple of 1024 bytes, the
+// period of the swizzle.
+__device__ __forceinline__ int swz(int o, int mask) { return o ^ (((o >> 7) & mask) << 4); }
+
+// Byte b of row r in a chunked box of nrows rows.
+__device__ __forceinline__ int box_off(int r, int nrows, int b) {
+  return swz(((b >> 7) * nrows + r) * 128 + (b & 127), 7);
 }
 
-// int8 m16 tile: rows g and g + 8 at ra / rb (K block kb at (kb - kb0) * 128),
-// zero rows where `valid` is false. The warp's K blocks kb = wi + KS j inside
-// [kb0, kb1) multiply B[j].
+// Swizzle mask of a scale box with S-byte rows (S a power of two, 16 .. 128).
+__host__ __device__ constexpr int scale_mask(int S) { return S >= 128 ? 7 : S / 16 - 1; }
+
+__host__ __device__ constexpr int align1k(int b) { return (b + 1023) / 1024 * 1024; }
+
+// K order of the MMA steps. In a 128-wide K block, 32-wide group q (one E8M0
+// scale per weight row) feeds two m16n8k16 steps h = 0, 1; lane quad member
+// t owns the group's elements 8 t .. 8 t + 7 and gives elements 8 t + 4 h +
+// {0, 1, 2, 3} to the step's logical columns 2t, 2t + 1, 2t + 8, 2t + 9 (A
+// and B alike). The B fragment of a K block is therefore, per q, the 8
+// activations 32 q + 8 t .. + 7 of token g: B[4 q .. 4 q + 3].
+
+// MXFP4 m16 tile: tile row g is row ra of code box ca, tile row g + 8 is row
+// rb of code box cb (both boxes of nrows rows); their E8M0 scales are rows ra
+// / rb of scale boxes sa / sb (S bytes per row). The warp's K blocks kb = wi
+// + KS j (j < NJ, kb < nkb) multiply B[j]. Each group's two MMAs start from
+// zero and the group's scales multiply the result into acc (fp32), so the
+// E2M1 operands need no scaling.
 template <int NJ, int KS>
-__device__ __forceinline__ void tile_s8(const char* ra, const char* rb, bool valid, int kb0, int kb1, int wi,
-                                        const uint32_t (&B)[NJ][16], float (&ae)[4], float (&ao)[4]) {
+__device__ __forceinline__ void tile_mx(const char* ca, int ra, const char* cb, int rb, int nrows, const char* sa,
+                                        const char* sb, int S, int wi, int nkb, const uint32_t (&B)[NJ][16],
+                                        float (&acc)[4]) {
+  const int t = threadIdx.x & 3;
+  const int sm = scale_mask(S);
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    const int kb = wi + KS * j;
+    if (kb < nkb) {
+      // the block's 4 group exponents of each row
+      const uint32_t ea = lds32(sa + swz(ra * S + 4 * kb, sm));
+      const uint32_t eb = lds32(sb + swz(rb * S + 4 * kb, sm));
+      const int la = (kb >> 1) * nrows + ra, lb = (kb >> 1) * nrows + rb;  // lines of the rows' chunk
+      const int u0 = (kb & 1) << 2;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t wa = lds32(ca + la * 128 + (((u0 + q) ^ (la & 7)) << 4) + 4 * t);
+        const uint32_t wb = lds32(cb + lb * 128 + (((u0 + q) ^ (lb & 7)) << 4) + 4 * t);
+        uint32_t xa[4], xb[4];
+        e2m1x8_to_f16x2(wa, xa);
+        e2m1x8_to_f16x2(wb, xb);
+        const uint32_t A0[4] = {xa[0], xb[0], xa[1], xb[1]};
+        const uint32_t A1[4] = {xa[2], xb[2], xa[3], xb[3]};
+        float d[4];
+        mma_16816_f16_zero(d, A0, B[j][4 * q], B[j][4 * q + 1]);
+        mma_16816_f16(d, A1, B[j][4 * q + 2], B[j][4 * q + 3]);
+        // E8M0 e is 2^(e - 127): the float with exponent field e
+        const float fa = __uint_as_float(((ea >> (8 * q)) & 0xFFu) << 23);
+        const float fb = __uint_as_float(((eb >> (8 * q)) & 0xFFu) << 23);
+        acc[0] = fmaf(d[0], fa, acc[0]);
+        acc[1] = fmaf(d[1], fa, acc[1]);
+        acc[2] = fmaf(d[2], fb, acc[2]);
+        acc[3] = fmaf(d[3], fb, acc[3]);
+      }
+    }
+  }
+}
+
+// int8 m16 tile: tile rows g / g + 8 are row ra of box ca / row rb of box cb
+// (chunked boxes of nrows rows), zero rows where `valid` is false; the warp's
+// K blocks kb = wi + KS j < nkb. Accumulates in ae (steps h = 0) and ao (h = 1).
+template <int NJ, int KS>
+__device__ __forceinline__ void tile_s8(const char* ca, int ra, const char* cb, int rb, int nrows, bool valid, int wi,
+                                        int nkb, const uint32_t (&B)[NJ][16], float (&ae)[4], float (&ao)[4]) {
   const int t = threadIdx.x & 3;
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
     const int kb = wi + KS * j;
-    if (kb >= kb0 && kb < kb1) {
-      uint4 qa0 = make_uint4(0u, 0u, 0u, 0u), qa1 = qa0, qb0 = qa0, qb1 = qa0;
-      if (valid) {
-        const char* pa = ra + (kb - kb0) * 128 + 32 * t;
-        const char* pb = rb + (kb - kb0) * 128 + 32 * t;
-        qa0 = *reinterpret_cast<const uint4*>(pa);
-        qa1 = *reinterpret_cast<const uint4*>(pa + 16);
-        qb0 = *reinterpret_cast<const uint4*>(pb);
-        qb1 = *reinterpret_cast<const uint4*>(pb + 16);
-      }
-      const uint32_t wa[8] = {qa0.x, qa0.y, qa0.z, qa0.w, qa1.x, qa1.y, qa1.z, qa1.w};
-      const uint32_t wb[8] = {qb0.x, qb0.y, qb0.z, qb0.w, qb1.x, qb1.y, qb1.z, qb1.w};
+    if (kb < nkb) {
+      const int la = kb * nrows + ra, lb = kb * nrows + rb;  // a K block is one chunk
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
+      for (int q = 0; q < 4; ++q) {
+        uint2 qa = make_uint2(0u, 0u), qb = qa;
+        if (valid) {
+          const int u = 2 * q + (t >> 1), w = 8 * (t & 1);
+          qa = lds64(ca + la * 128 + ((u ^ (la & 7)) << 4) + w);
+          qb = lds64(cb + lb * 128 + ((u ^ (lb & 7)) << 4) + w);
+        }
         uint32_t A[4];
-        s8x4_to_f16x2(wa[s], A[0], A[2]);
-        s8x4_to_f16x2(wb[s], A[1], A[3]);
-        if (s & 1)
-          mma_16816_f16(ao, A, B[j][2 * s], B[j][2 * s + 1]);
-        else
-          mma_16816_f16(ae, A, B[j][2 * s], B[j][2 * s + 1]);
+        s8x4_to_f16x2(qa.x, A[0], A[2]);
+        s8x4_to_f16x2(qb.x, A[1], A[3]);
+        mma_16816_f16(ae, A, B[j][4 * q], B[j][4 * q + 1]);
+        s8x4_to_f16x2(qa.y, A[0], A[2]);
+        s8x4_to_f16x2(qb.y, A[1], A[3]);
+        mma_16816_f16(ao, A, B[j][4 * q + 2], B[j][4 * q + 3]);
       }
     }
+  }
+}
+
+// B fragments of K block kb for token row `row` (f16 elements, K block at kb
+// * 128): per group q the 8 activations 32 q + 8 t .. + 7.
+__device__ __forceinline__ void load_b_smem(const char* row, int kb, uint32_t (&B)[16]) {
+  const int t = threadIdx.x & 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 v = lds128(row + (kb * 128 + 32 * q + 8 * t) * 2);
+    B[4 * q] = v.x;
+    B[4 * q + 1] = v.y;
+    B[4 * q + 2] = v.z;
+    B[4 * q + 3] = v.w;
   }
 }
 
@@ -326,7 +390,7 @@ __device__ __forceinline__ void route_tables(RouteSmem& S, Tables& tb, const Dec
 }
 
 // The tables, for the w2 kernel (one warp).
-__device__ __noinline__ void publish_tables(const Tables& tb, const DecParams& P) {
+__device__ __forceinline__ void publish_tables(const Tables& tb, const DecParams& P) {
   const int lane = threadIdx.x & 31;
   for (int i = lane; i < tb.nh; i += 32) {
     P.ctl[cHit + i] = uint32_t(tb.hit[i]);
@@ -338,7 +402,7 @@ __device__ __noinline__ void publish_tables(const Tables& tb, const DecParams& P
 
 // Stable counting sort of the batch's slots by expert (layer-mode outputs),
 // from the state route_tables left in shared memory; one warp.
-__device__ __noinline__ void write_permutation(RouteSmem& S, const DecParams& P, int nh) {
+__device__ __forceinline__ void write_permutation(RouteSmem& S, const DecParams& P, int nh) {
   const int lane = threadIdx.x & 31;
   const int Sn = P.T * P.k;
   const int c0 = 2 * lane < nh ? S.cnt[2 * lane] : 0;
@@ -476,24 +540,26 @@ __device__ __forceinline__ Item w13_item(const DecParams& P, const Tables& tb, i
   return m;
 }
 
-// Copies slab m into stage s (lane 0 of the calling warp issues and arms).
-__device__ __forceinline__ void fill13(const DecParams& P, W13Smem& S, char* dst, int s, const Item& m, int pos) {
+// Copies slab m into stage s (lane 0 of the calling warp issues and arms):
+// routed, the gate and up code boxes (8 rows each) and their scale boxes;
+// shared, the 4 gate and 4 up int8 rows as two boxes.
+__device__ __forceinline__ void fill13(const DecParams& P, const DecMaps& M, W13Smem& S, char* dst, int s,
+                                       const Item& m, int pos) {
   const int H = P.H;
   if ((threadIdx.x & 31) == 0) {
     S.lastfill[s] = pos;
     if (m.kind == kS13) {
-      const char* sh = reinterpret_cast<const char*>(P.sh13);
       mbar_arrive_expect_tx(&S.full[s], uint32_t(8 * H));
-      bulk_g2s(dst, sh + size_t(m.row0) * H, uint32_t(4 * H), &S.full[s]);
-      bulk_g2s(dst + 4 * H, sh + size_t(P.Is + m.row0) * H, uint32_t(4 * H), &S.full[s]);
+      tma_load_3d(dst, &M.shared, 0, m.row0, 0, &S.full[s]);
+      tma_load_3d(dst + 4 * H, &M.shared, 0, P.Is + m.row0, 0, &S.full[s]);
     } else {
-      const size_t rg = size_t(m.e) * 2 * P.I + m.row0, ru = rg + P.I;
-      mbar_arrive_expect_tx(&S.full[s], uint32_t(16 * (H / 2) + 16 * (H / 32)));
-      bulk_g2s(dst, P.w13_codes + rg * (H / 2), uint32_t(8 * (H / 2)), &S.full[s]);
-      bulk_g2s(dst + 8 * (H / 2), P.w13_codes + ru * (H / 2), uint32_t(8 * (H / 2)), &S.full[s]);
-      bulk_g2s(dst + 16 * (H / 2), P.w13_scales + rg * (H / 32), uint32_t(8 * (H / 32)), &S.full[s]);
-      bulk_g2s(dst + 16 * (H / 2) + 8 * (H / 32), P.w13_scales + ru * (H / 32), uint32_t(8 * (H / 32)),
-               &S.full[s]);
+      const int rg = m.e * 2 * P.I + m.row0, ru = rg + P.I;
+      const int sc = 8 * H, sbox = align1k(8 * (H / 32));
+      mbar_arrive_expect_tx(&S.full[s], uint32_t(8 * H + 16 * (H / 32)));
+      tma_load_3d(dst, &M.codes, 0, rg, 0, &S.full[s]);
+      tma_load_3d(dst + 4 * H, &M.codes, 0, ru, 0, &S.full[s]);
+      tma_load_2d(dst + sc, &M.scales, 0, rg, &S.full[s]);
+      tma_load_2d(dst + sc + sbox, &M.scales, 0, ru, &S.full[s]);
     }
   }
   __syncwarp();
@@ -537,7 +603,7 @@ __device__ __forceinline__ void prefetch_w2_share(const DecParams& P, const Tabl
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
+__global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P, const __grid_constant__ DecMaps M) {
   extern __shared__ __align__(128) char smem[];
   W13Smem& S = *reinterpret_cast<W13Smem*>(smem);
   // Test hook (word 1 of the status block, zero in normal use): a wait on a
@@ -551,7 +617,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
     }
     return;
   }
-  char* stages = smem + kHead13;
+  // stages at the next multiple of 1024 bytes (the swizzle's period)
+  char* stages = smem + ((smem_u32(smem) + uint32_t(kHead13) + 1023u) & ~1023u) - smem_u32(smem);
   float4* parts = reinterpret_cast<float4*>(stages + size_t(kStages13) * P.stage_bytes);
   // router scores and bias, outside the ring (it takes the shared slabs
   // before the routing is known)
@@ -616,10 +683,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
     for (int j = 0; j < kNJ; ++j) {
       const int kb = wi + 8 * j;
       if (kb < nkbH && g < T) {
-        const uint4* src = reinterpret_cast<const uint4*>(P.x + size_t(g) * H + kb * 128 + 32 * t);
+        // group p: activations kb * 128 + 32 p + 8 t .. + 7 (the MMA steps' K order)
+        const __nv_bfloat16* src = P.x + size_t(g) * H + kb * 128 + 8 * t;
   #pragma unroll
         for (int p = 0; p < 4; ++p) {
-          const uint4 v = __ldg(src + p);
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + 32 * p));
           B[j][4 * p] = v.x;
           B[j][4 * p + 1] = v.y;
           B[j][4 * p + 2] = v.z;
@@ -634,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
   __syncthreads();
   if (warp == 14)
     for (int p = 0; p < nsp; ++p)
-      fill13(P, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, c0.s0 + p), p);
+      fill13(P, M, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, c0.s0 + p), p);
   if (q == 1 && gt < nsr) {
     S.sh_scale[0][gt] = rsg;
     S.sh_scale[1][gt] = rsu;
@@ -679,19 +747,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
   auto run_item = [&](const Chunk& ch, int npos, int pos, bool refill, bool need_tables) -> bool {
     const Item m = w13_item(P, S.tb, ch.item(pos, n_s));
     const int s = pos % kStages13;
-    if (!__all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / kStages13) & 1u, P))) return false;
+    if (!__all_sync(0xffffffffu, wait_stage(&S.full[s], &S.lastfill[s], pos, kStages13, P))) return false;
     const char* st = stages + size_t(s) * P.stage_bytes;
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
     float4 p0;
     if (m.kind == kR13) {
-      const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + 16 * (H / 2));
-      float fa, fb;
-      tile_mx<kNJ, 8>(st + g * (H / 2), st + (g + 8) * (H / 2), sc + g * (H / 32), sc + (g + 8) * (H / 32), wi,
-                      nkbH, B, a0, a1, fa, fb);
-      p0 = make_float4((a0[0] + a1[0]) * fa, (a0[1] + a1[1]) * fa, (a0[2] + a1[2]) * fb, (a0[3] + a1[3]) * fb);
+      // gate rows (tile rows g) and up rows (g + 8): code boxes at 0 and 4H,
+      // their scale boxes from 8H
+      const char* sc = st + 8 * H;
+      tile_mx<kNJ, 8>(st, g, st + 4 * H, g, 8, sc, sc + align1k(8 * (H / 32)), H / 32, wi, nkbH, B, a0);
+      p0 = make_float4(a0[0], a0[1], a0[2], a0[3]);
     } else {
       // rows g < 4: gate row g of the slab (tile row g) and up row g (tile row g + 8)
-      tile_s8<kNJ, 8>(st + (g & 3) * H, st + (4 + (g & 3)) * H, g < 4, 0, nkbH, wi, B, a0, a1);
+      tile_s8<kNJ, 8>(st, g & 3, st + 4 * H, g & 3, 4, g < 4, wi, nkbH, B, a0, a1);
       p0 = make_float4(a0[0] + a1[0], a0[1] + a1[1], a0[2] + a1[2], a0[3] + a1[3]);
     }
     float4* part = parts + size_t(s) * kGW * 32;
@@ -729,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
         nr = cr.size();
       }
       if (have && pos + kStages13 < nr) {
-        fill13(P, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, cr.item(pos + kStages13, n_s)),
+        fill13(P, M, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, cr.item(pos + kStages13, n_s)),
                pos + kStages13);
         if (pos + kStages13 == nr - 1 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
       }
@@ -790,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P) {
       const Chunk cr = w13_chunk(P, S.tb.nh, b, G);
       const int nr = cr.size();
       for (int p = nsp; p < kStages13 && p < nr; ++p)
-        fill13(P, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, cr.item(p, n_s)), p);
+        fill13(P, M, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, cr.item(p, n_s)), p);
       if (nr <= kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
       __threadfence_block();
       if (lane == 0) *reinterpret_cast<volatile int*>(&S.ready) = 1;
@@ -854,22 +922,26 @@ __device__ __forceinline__ Item2 w2_item(const DecParams& P, int nl, int b, int 
   return m;
 }
 
-// Offset of the token rows of intermediates in a stage.
-__device__ __forceinline__ int w2_hoff(const DecParams& P) {
-  return max(16 * P.Is, 16 * (P.I / 2) + 16 * (P.I / 32));
+// Offset of the token rows of intermediates in a stage: after the larger of
+// the shared box (16 int8 rows) and the routed code box (16 rows of I / 2
+// bytes) with its scale box.
+__host__ __device__ __forceinline__ int w2_hoff(int I, int Is) {
+  const int sh = 16 * Is, ro = 8 * I + align1k(16 * (I / 32));
+  return align1k(sh > ro ? sh : ro);
 }
 
-// Weight rows [rb * 16, +16) of the item's expert: adds their bytes to the
-// stage's barrier without arriving (lane 0).
-__device__ __forceinline__ void fill2_weights(const DecParams& P, W2Smem& S, char* dst, int s, const Item2& m) {
+// Weight rows [rb * 16, +16) of the item's expert as one code box (and its
+// scale box): adds their bytes to the stage's barrier without arriving (lane 0).
+__device__ __forceinline__ void fill2_weights(const DecParams& P, const DecMaps& M, W2Smem& S, char* dst, int s,
+                                              const Item2& m) {
   if (m.li < 0) {
     mbar_expect_tx(&S.full[s], uint32_t(16 * P.Is));
-    bulk_g2s(dst, reinterpret_cast<const char*>(P.sh2) + size_t(m.rb) * 16 * P.Is, uint32_t(16 * P.Is), &S.full[s]);
+    tma_load_3d(dst, &M.shared, 0, m.rb * 16, 0, &S.full[s]);
   } else {
-    const size_t r0 = size_t(S.tb.hit[m.li]) * P.H + size_t(m.rb) * 16;
+    const int r0 = S.tb.hit[m.li] * P.H + m.rb * 16;
     mbar_expect_tx(&S.full[s], uint32_t(16 * (P.I / 2) + 16 * (P.I / 32)));
-    bulk_g2s(dst, P.w2_codes + r0 * (P.I / 2), uint32_t(16 * (P.I / 2)), &S.full[s]);
-    bulk_g2s(dst + 16 * (P.I / 2), P.w2_scales + r0 * (P.I / 32), uint32_t(16 * (P.I / 32)), &S.full[s]);
+    tma_load_3d(dst, &M.codes, 0, r0, 0, &S.full[s]);
+    tma_load_2d(dst + 8 * P.I, &M.scales, 0, r0, &S.full[s]);
   }
 }
 
@@ -884,15 +956,15 @@ __device__ __forceinline__ void fill2_h(const DecParams& P, W2Smem& S, char* dst
   __syncwarp();
   if (lane < P.T && ((mask >> lane) & 1u)) {
     const __half* src = sh ? P.hs + size_t(lane) * P.Is : P.dh + (size_t(m.li) * P.T + lane) * P.I;
-    bulk_g2s(dst + w2_hoff(P) + lane * K * 2, src, uint32_t(K * 2), &S.full[s]);
+    bulk_g2s(dst + w2_hoff(P.I, P.Is) + lane * K * 2, src, uint32_t(K * 2), &S.full[s]);
   }
   __syncwarp();
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
+__global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P, const __grid_constant__ DecMaps M) {
   extern __shared__ __align__(128) char smem[];
   W2Smem& S = *reinterpret_cast<W2Smem*>(smem);
-  char* stages = smem + kHead2;
+  char* stages = smem + ((smem_u32(smem) + uint32_t(kHead2) + 1023u) & ~1023u) - smem_u32(smem);
   float4* red = reinterpret_cast<float4*>(stages + size_t(P.nstages) * P.stage_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -915,7 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
     fence_mbar_init();
     // Position 0 is the shared expert of the first block: its weight rows do
     // not depend on the previous grids.
-    if (has_sh && nrb_mine > 0) fill2_weights(P, S, stages, 0, Item2{b * P.w2_per, 0, -1});
+    if (has_sh && nrb_mine > 0) fill2_weights(P, M, S, stages, 0, Item2{b * P.w2_per, 0, -1});
   }
   __syncthreads();
   pdl_wait();
@@ -928,7 +1000,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
       const Item2 m = w2_item(P, nl, b, p);
       if (lane == 0) {
         S.lastfill[p] = p;
-        if (!(p == 0 && has_sh)) fill2_weights(P, S, stages + size_t(p) * P.stage_bytes, p, m);
+        if (!(p == 0 && has_sh)) fill2_weights(P, M, S, stages + size_t(p) * P.stage_bytes, p, m);
       }
       __syncwarp();
       fill2_h(P, S, stages + size_t(p) * P.stage_bytes, p, m);
@@ -954,7 +1026,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
       const int s = pos % NS;
       // A timed-out warp keeps going (without reading the stage) so that every
       // warp reaches the block-end barriers.
-      ok = ok && __all_sync(0xffffffffu, wait_bar(&S.full[s], uint32_t(pos / NS) & 1u, P));
+      ok = ok && __all_sync(0xffffffffu, wait_stage(&S.full[s], &S.lastfill[s], pos, NS, P));
       if (!ok) continue;
       const char* st = stages + size_t(s) * P.stage_bytes;
       const bool sh = m.li < 0;
@@ -968,15 +1040,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
       for (int j = 0; j < 2; ++j) {
         const int kb = wi + 8 * j;
         if (has_tok && kb < nkb) {
-          const uint4* p4 = reinterpret_cast<const uint4*>(st + w2_hoff(P) + g * K * 2 + kb * 256 + 64 * t);
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const uint4 v = p4[p];
-            Bf[j][4 * p] = v.x;
-            Bf[j][4 * p + 1] = v.y;
-            Bf[j][4 * p + 2] = v.z;
-            Bf[j][4 * p + 3] = v.w;
-          }
+          load_b_smem(st + w2_hoff(P.I, P.Is) + g * K * 2, kb, Bf[j]);
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i) Bf[j][i] = 0u;
@@ -984,7 +1048,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
       }
       float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
       if (sh) {
-        tile_s8<2, 8>(st + g * P.Is, st + (g + 8) * P.Is, true, 0, nkb, wi, Bf, a0, a1);
+        tile_s8<2, 8>(st, g, st, g + 8, 16, true, wi, nkb, Bf, a0, a1);
         const int rl = (m.rb - b * P.w2_per) * 16 + g;  // row within this CTA's output rows
         const float its = 1.0f / P.tau_s;
         const float sa = (rl < kShRows ? S.sh_scale[rl] : __ldg(P.sh2_scale + m.rb * 16 + g)) * its;
@@ -994,16 +1058,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
         acc.z += (a0[2] + a1[2]) * sb;
         acc.w += (a0[3] + a1[3]) * sb;
       } else {
-        const int rs = P.I / 2, Gs = P.I / 32;
-        const uint8_t* sc = reinterpret_cast<const uint8_t*>(st + 16 * rs);
-        float fa, fb;
-        tile_mx<2, 8>(st + g * rs, st + (g + 8) * rs, sc + g * Gs, sc + (g + 8) * Gs, wi, nkb, Bf, a0, a1, fa, fb);
-        fa *= 1.0f / P.tau_r;
-        fb *= 1.0f / P.tau_r;
-        acc.x += (a0[0] + a1[0]) * fa;
-        acc.y += (a0[1] + a1[1]) * fa;
-        acc.z += (a0[2] + a1[2]) * fb;
-        acc.w += (a0[3] + a1[3]) * fb;
+        const char* sc = st + 8 * P.I;  // the scale box after the 16-row code box
+        tile_mx<2, 8>(st, g, st, g + 8, 16, sc, sc, P.I / 32, wi, nkb, Bf, a0);
+        const float itr = 1.0f / P.tau_r;
+        acc.x += a0[0] * itr;
+        acc.y += a0[1] * itr;
+        acc.z += a0[2] * itr;
+        acc.w += a0[3] * itr;
       }
       // the last warp of the group to finish with the stage refills it
       __syncwarp();
@@ -1018,7 +1079,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P) {
           const Item2 mn = w2_item(P, nl, b, np);
           if (lane == 0) {
             S.lastfill[s] = np;
-            fill2_weights(P, S, stages + size_t(s) * P.stage_bytes, s, mn);
+            fill2_weights(P, M, S, stages + size_t(s) * P.stage_bytes, s, mn);
           }
           __syncwarp();
           fill2_h(P, S, stages + size_t(s) * P.stage_bytes, s, mn);
@@ -1074,20 +1135,51 @@ Plan make_plan(const v4moe_config& c, int T) {
   if (T < 1 || T > kDecodeMaxTokens || T * c.top_k > kMaxHit) return p;
   const int H = c.hidden, I = c.inter, Is = c.shared_inter;
   if (H > kNJ * 8 * 128 || I > 2 * 8 * 128 || Is > 2 * 8 * 128) return p;
-  int s13 = 16 * (H / 2) + 16 * (H / 32);
-  if (Is > 0) s13 = std::max(s13, 8 * H);
-  p.stage13 = (s13 + 127) / 128 * 128;
+  // Scale rows of K / 32 bytes: a swizzle span (16 .. 128 bytes), so K is a
+  // power of two from 512; shared rows whole 128-byte chunks.
+  auto pow2 = [](int v) { return v > 0 && (v & (v - 1)) == 0; };
+  if (H % 512 != 0 || I % 512 != 0 || !pow2(H) || !pow2(I) || Is % 128 != 0) return p;
+  const int s13 = std::max(8 * H + 2 * align1k(8 * (H / 32)), Is > 0 ? 8 * H : 0);
+  p.stage13 = align1k(s13);
   const size_t route_stage = (size_t(T) * c.n_experts + c.n_experts) * 4;  // scores + bias
-  p.smem13 = kHead13 + size_t(kStages13) * p.stage13 + kPart13 + (route_stage + 127) / 128 * 128;
-  const int hoff = std::max(16 * Is, 16 * (I / 2) + 16 * (I / 32));
-  const int s2 = hoff + T * std::max(I, Is) * 2;
-  p.stage2 = (s2 + 127) / 128 * 128;
-  const size_t room = 227 * 1024 - kHead2 - kRed2;
+  // 1024 bytes of slack put the first stage on a multiple of 1024
+  p.smem13 = kHead13 + 1024 + size_t(kStages13) * p.stage13 + kPart13 + (route_stage + 127) / 128 * 128;
+  p.stage2 = align1k(w2_hoff(I, Is) + T * std::max(I, Is) * 2);
+  const size_t room = 227 * 1024 - kHead2 - 1024 - kRed2;
   p.nst2 = int(std::min<size_t>(kMaxStages2, room / p.stage2));
-  p.smem2 = kHead2 + size_t(p.nst2) * p.stage2 + kRed2;
-  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 &&
-         size_t(T) * H * 2 <= 227 * 1024;
+  p.smem2 = kHead2 + 1024 + size_t(p.nst2) * p.stage2 + kRed2;
+  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 && size_t(T) * H * 2 <= 227 * 1024;
   return p;
+}
+
+// u8 maps of the weights the slab kernels stream (see DecMaps). False when a
+// map cannot be encoded (a base address off 16 bytes).
+bool dec_maps(const v4moe_config& c, const v4moe_weights& w, DecMaps& m13, DecMaps& m2) {
+  const uint64_t H = c.hidden, I = c.inter, Is = c.shared_inter, E = c.n_experts;
+  auto chunked = [](CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+    const uint64_t dims[3] = {128, rows, row_bytes / 128};
+    const uint64_t strides[2] = {row_bytes, 128};
+    const uint32_t box[3] = {128, box_rows, uint32_t(row_bytes / 128)};
+    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+  };
+  auto scales = [](CUtensorMap* m, const void* base, uint64_t rows, uint64_t S, uint32_t box_rows) {
+    const uint64_t dims[2] = {S, rows};
+    const uint64_t strides[1] = {S};
+    const uint32_t box[2] = {uint32_t(S), box_rows};
+    const CUtensorMapSwizzle sw = S >= 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : S == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : S == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                            : CU_TENSOR_MAP_SWIZZLE_NONE;
+    return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, sw);
+  };
+  m13 = DecMaps{};
+  m2 = DecMaps{};
+  bool ok = chunked(&m13.codes, w.w13_codes, E * 2 * I, H / 2, 8) && scales(&m13.scales, w.w13_scales, E * 2 * I, H / 32, 8) &&
+            chunked(&m2.codes, w.w2_codes, E * H, I / 2, 16) && scales(&m2.scales, w.w2_scales, E * H, I / 32, 16);
+  if (ok && Is > 0)
+    ok = chunked(&m13.shared, w.sh_w13, 2 * Is, H, 4) && chunked(&m2.shared, w.sh_w2, H, Is, 16);
+  return ok;
 }
 
 }  // namespace
@@ -1107,6 +1199,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const v4moe_config& c = a.c;
   const Plan p = make_plan(c, a.T);
   if (!p.ok) return cudaErrorInvalidValue;
+  DecMaps m13, m2;
+  if (!dec_maps(c, a.w, m13, m2)) return cudaErrorInvalidValue;
   const int sms = device_sms();
   DecParams P;
   P.T = a.T;
@@ -1169,12 +1263,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   // previous call's w2 kernel (it rewrites the intermediates that one reads).
   P.stage_bytes = p.stage13;
   set_smem(k_dec_w13, p.smem13);
-  e = launch_kernel("dec_w13", k_dec_w13, dim3(sms), dim3(kThreads), p.smem13, st, a.layer_mode != 0, P);
+  e = launch_kernel("dec_w13", k_dec_w13, dim3(sms), dim3(kThreads), p.smem13, st, a.layer_mode != 0, P, m13);
   if (e != cudaSuccess) return e;
   P.stage_bytes = p.stage2;
   P.nstages = p.nst2;
   set_smem(k_dec_w2, p.smem2);
-  return launch_kernel("dec_w2", k_dec_w2, dim3(grid2), dim3(kThreads), p.smem2, st, true, P);
+  return launch_kernel("dec_w2", k_dec_w2, dim3(grid2), dim3(kThreads), p.smem2, st, true, P, m2);
 }
 
 }  // namespace v4moe

@@ -291,14 +291,6 @@ __device__ __forceinline__ MxGeo mx_geo(const MxParams& P, const MxTile& t, int 
   return g;
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
-          smem_u32(dst)),
-      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Instruction descriptor of kind::mxf8f6f4 with E2M1 A, E4M3 B, E8M0 scales,
 // both operands K-major: A format bits 7-9 = 5, B format bits 10-12 = 0,
 // N >> 3 at bits 17-22, scale format bit 23 = 1 (E8M0), M >> 4 at bits 24-28;

@@ -1,6 +1,7 @@
 // Internal declarations shared by the libv4moe translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -29,6 +30,14 @@ constexpr int kPermChunk = 2048;
 bool config_ok(const v4moe_config* c);
 int32_t check_device();
 int device_sms();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link to
+// libcuda): a tiled map of rank 2 or 3 with unit element strides, no
+// interleave, L2 promotion of 256 bytes and no fill. dims / box list the
+// innermost dimension first; strides[i] is the byte stride of dimension i + 1.
+// False when the entry point is missing or the driver rejects the map.
+bool encode_tensor_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                       const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw);
 
 size_t tc_extra_bytes(const v4moe_config& c, int64_t T);
 
