@@ -14,24 +14,22 @@
 // Kernels:
 //  * k_dec_route: router scores (one warp per expert); the last CTA to finish
 //    selects each token's experts and publishes the batch's routing tables
-//    (distinct experts in ascending id, token masks, weights) and the
-//    permutation outputs. In forward mode one CTA publishes the tables of the
-//    caller's routing.
+//    (distinct experts in ascending id, token masks, weights), the routing
+//    outputs and the permutation.
 //  * k_dec_w13: one CTA per SM, two groups of eight warps. Work items are w13
 //    slabs (8 channels of a routed expert: 8 gate rows and the 8 matching up
 //    rows; or 4 + 4 int8 rows of the shared expert), numbered shared first,
 //    then routed expert by expert; CTA b takes a contiguous share of each as
-//    its ring positions 0, 1, .... The shared slabs do not depend on the
-//    routing: their copies are issued at the start and group 1 multiplies
-//    them while group 0 selects from the router's scores and builds the
-//    routing tables; then both groups take alternate positions of the routed
-//    slabs, and once its last slab is on its way the CTA asks L2 for its
-//    share of the routed w2 rows. Warp i of a group owns the 128-wide K
-//    blocks i, i + 8, ... of a slab, multiplies them by the activations with
-//    mma.sync m16n8k16 (f16 operands, fp32 accumulation, the tokens as the 8
-//    columns) and posts its partial tile to shared memory; the last warp to
-//    post sums the partials in warp order, refills the stage and writes h as
-//    f16 (routed: w * h).
+//    its ring positions 0, 1, ..., and group q the positions q, q + 2, ....
+//    A CTA reads x, its row scales and the routing tables (in forward mode it
+//    builds the tables from the caller's routing) before its first copy, and
+//    once its last slab is on its way asks L2 for its share of the routed w2
+//    rows. Warp i of a group owns the 128-wide K blocks i, i + 8, ... of a
+//    slab, multiplies them by the activations with mma.sync m16n8k16 (f16
+//    operands, fp32 accumulation, the tokens as the 8 columns) and posts its
+//    partial tile to shared memory; the last warp to post sums the partials
+//    in warp order, refills the stage and stages h as f16 (routed: w * h) in
+//    shared memory; the CTA writes its h rows once its slabs are done.
 //  * k_dec_w2: two groups of eight warps, warp i of a group owning K blocks
 //    i, i + 8. CTA b owns a run of 16-row output blocks and goes through the
 //    shared expert and every routed expert for each of them, the two groups
@@ -65,6 +63,8 @@
 
 #include <algorithm>
 #include <cmath>
+#include <map>
+#include <mutex>
 
 #include "launch.cuh"
 #include "ptx.cuh"
@@ -101,6 +101,7 @@ struct DecParams {
   int stage_bytes;
   int nstages;  // w2 ring depth
   int w2_per;   // 16-row output blocks per w2 CTA
+  int hrs, hss;  // w13: per-token row capacity of the staged routed / shared intermediates
   const __nv_bfloat16* x;
   const __nv_bfloat16* gate;
   const float* bias;
@@ -187,12 +188,12 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t w) {
 
 // Whole CTA; the caller synchronises afterwards.
 __device__ __forceinline__ void read_tables(Tables& tb, const DecParams& P) {
-  const int nh = int(P.ctl[cNh]);
+  const int nh = int(__ldcg(P.ctl + cNh));
   for (int i = threadIdx.x; i < nh; i += blockDim.x) {
-    tb.hit[i] = int(P.ctl[cHit + i]);
-    tb.mask[i] = P.ctl[cMask + i];
+    tb.hit[i] = int(__ldcg(P.ctl + cHit + i));
+    tb.mask[i] = __ldcg(P.ctl + cMask + i);
   }
-  for (int i = threadIdx.x; i < nh * 8; i += blockDim.x) tb.w[i] = reinterpret_cast<const float*>(P.ctl + cW)[i];
+  for (int i = threadIdx.x; i < nh * 8; i += blockDim.x) tb.w[i] = __ldcg(reinterpret_cast<const float*>(P.ctl + cW) + i);
   if (threadIdx.x == 0) tb.nh = nh;
 }
 
@@ -208,11 +209,6 @@ __device__ __forceinline__ void read_tables(Tables& tb, const DecParams& P) {
 // S (none at 16 bytes). Every box starts at a multiple of 1024 bytes, the
 // period of the swizzle.
 __device__ __forceinline__ int swz(int o, int mask) { return o ^ (((o >> 7) & mask) << 4); }
-
-// Byte b of row r in a chunked box of nrows rows.
-__device__ __forceinline__ int box_off(int r, int nrows, int b) {
-  return swz(((b >> 7) * nrows + r) * 128 + (b & 127), 7);
-}
 
 // Swizzle mask of a scale box with S-byte rows (S a power of two, 16 .. 128).
 __host__ __device__ constexpr int scale_mask(int S) { return S >= 128 ? 7 : S / 16 - 1; }
@@ -439,63 +435,157 @@ __device__ __forceinline__ void write_permutation(RouteSmem& S, const DecParams&
   }
 }
 
-// Top-k selection of token t (one warp) from scores and bias in shared memory,
-// into the RouteSmem selection arrays. Inlined: the routing runs while the
-// shared slabs' copies are in flight, and on this GPU the local-memory traffic
-// of a call (saved registers) would wait behind them.
-__device__ __forceinline__ void select_token(RouteSmem& S, const DecParams& P, int t, const float* ssc,
-                                             const float* sbias) {
-  if (P.token_ids)
-    select_hash_warp<true>(t, P.E, P.k, P.vocab, P.routed_scale, ssc + size_t(t) * P.E, P.token_ids, P.tid2eid,
-                           S.sel_ids, S.sel_w, P.status);
-  else if (P.E <= 256)
-    select_learned_n<false, 8>(t, P.E, P.k, P.routed_scale, ssc + size_t(t) * P.E, sbias, S.sel_ids, S.sel_w);
-  else
-    select_learned_n<false, 32>(t, P.E, P.k, P.routed_scale, ssc + size_t(t) * P.E, sbias, S.sel_ids, S.sel_w);
+constexpr int kRouteWarps = 16;
+constexpr int kRouteMaxCluster = 16;
+
+// Learned routing of token t by one warp from E <= 32 NPER scores s and bias b
+// in shared memory: k rounds of a warp arg-max over s + b (larger key, then
+// lower id), then the k winners ordered by id and w = scale * s / (their sum
+// in that order) -- the same selection, ties and rounding as
+// select_learned_n, written as loops: the router runs it once per call with
+// its instructions not yet in any cache, so its length is its latency.
+template <int NPER>
+__device__ __noinline__ void select_compact(int t, int E, int k, float scale, const float* s, const float* b,
+                                            int32_t* ids, float* w) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[NPER];  // 0: not an expert, or already taken
+#pragma unroll
+  for (int i = 0; i < NPER; ++i) {
+    const int e = lane + 32 * i;
+    float v = 0.f;
+    if (e < E) v = s[e] + b[e];
+    key[i] = e < E ? float_key(v != v ? -INFINITY : v) : 0u;
+  }
+  int myid = 0x7fffffff;  // lane r < k: the winner of round r
+  float myv = 0.f;
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    uint32_t lk = 0u;
+    int li = 0;
+#pragma unroll
+    for (int i = 0; i < NPER; ++i)
+      if (key[i] > lk) {  // strict: the lowest id among equal keys
+        lk = key[i];
+        li = i;
+      }
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, lk);
+    const uint32_t cand = (lk == mk && lk != 0u) ? uint32_t(lane + 32 * li) : 0xffffffffu;
+    const uint32_t wid = __reduce_min_sync(0xffffffffu, cand);
+    if (lane == int(wid & 31u))
+#pragma unroll
+      for (int i = 0; i < NPER; ++i)
+        if (i == int(wid >> 5)) key[i] = 0u;
+    if (lane == r) {
+      myid = int(wid);
+      myv = wid < uint32_t(E) ? s[wid] : 0.f;
+    }
+  }
+  int rank = 0;  // position of this lane's winner in ascending id order
+#pragma unroll 1
+  for (int j = 0; j < k; ++j) rank += __shfl_sync(0xffffffffu, myid, j) < myid;
+  float sum = 0.f;
+#pragma unroll 1
+  for (int p = 0; p < k; ++p) {
+    const unsigned m = __ballot_sync(0xffffffffu, lane < k && rank == p);
+    sum += __shfl_sync(0xffffffffu, myv, __ffs(m) - 1);
+  }
+  if (lane < k) {
+    ids[size_t(t) * k + rank] = myid;
+    w[size_t(t) * k + rank] = scale * (myv / sum);
+  }
 }
 
-constexpr int kRouteWarps = 8;
+// What the router's leader CTA keeps in shared memory besides the scores.
+struct RouteTail {
+  RouteSmem rt;
+  Tables tb;
+};
+constexpr size_t kRouteTail = (sizeof(RouteTail) + 15) / 16 * 16;
 
-// Router scores s[t, e] (one warp per expert, the x rows staged in shared
-// memory). The selection happens in every CTA of the next kernel.
+// Router: one thread-block cluster of CL CTAs. Warp w of CTA r scores experts
+// e = r * kRouteWarps + w, + CL * kRouteWarps, ... (one warp per expert, the
+// x rows staged in shared memory) and stores s[t, e] into the leader CTA's
+// shared memory; after the cluster barrier the leader (rank 0) selects each
+// token's experts (bias prefetched into its shared memory), builds the
+// batch's routing tables (distinct experts in ascending id, token masks,
+// weights) and writes them for the slab kernels, with the routing outputs and
+// the permutation. Shared memory: tail, scores [T][E], bias [E], x [T][H].
 __global__ void __launch_bounds__(kRouteWarps * 32) k_dec_route(DecParams P) {
   extern __shared__ __align__(16) char rsm[];
-  // The w13 kernel may start now: before it waits for this grid it only reads
-  // the activations and asks L2 for weights.
-  pdl_launch_dependents();
+  RouteTail& R = *reinterpret_cast<RouteTail*>(rsm);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = P.H, T = P.T, E = P.E;
-  uint4* xs = reinterpret_cast<uint4*>(rsm);
-  const int e = blockIdx.x * kRouteWarps + warp;
-  // the whole gate row in flight at once (H <= 4096: up to 16 pieces per lane)
-  const uint4* grow = reinterpret_cast<const uint4*>(P.gate + size_t(e < E ? e : 0) * H);
+  float* sc = reinterpret_cast<float*>(rsm + kRouteTail);
+  float* sb = sc + size_t(T) * E;
+  uint4* xs = reinterpret_cast<uint4*>(rsm + kRouteTail + ((size_t(T) * E + E) * 4 + 15) / 16 * 16);
+  const uint32_t rank = cluster_ctarank();
+  const int CL = int(gridDim.x);
+  // The w13 kernel may start now: before it waits for this grid it reads only
+  // the activations and weights and issues its shared-expert copies.
+  pdl_launch_dependents();
   const int np = H / 8 / 32;
+  int e = int(rank) * kRouteWarps + warp;
+  // the first gate row in flight at once (H <= 4096: up to 16 pieces per lane)
   uint4 gv[16];
+  {
+    const uint4* grow = reinterpret_cast<const uint4*>(P.gate + size_t(e < E ? e : 0) * H);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) gv[i] = i < np ? __ldg(grow + lane + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
-  for (int i = threadIdx.x; i < T * H / 8; i += blockDim.x) xs[i] = __ldg(reinterpret_cast<const uint4*>(P.x) + i);
-  __syncthreads();
-  if (e >= E) return;
-  for (int t = 0; t < T; ++t) {
-    const uint4* xrow = xs + size_t(t) * (H / 8);
-    float acc = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (i < np) {
-        const uint4 xv = xrow[lane + 32 * i];
-        acc = fmaf(bf16_lo(gv[i].x), bf16_lo(xv.x), acc);
-        acc = fmaf(bf16_hi(gv[i].x), bf16_hi(xv.x), acc);
-        acc = fmaf(bf16_lo(gv[i].y), bf16_lo(xv.y), acc);
-        acc = fmaf(bf16_hi(gv[i].y), bf16_hi(xv.y), acc);
-        acc = fmaf(bf16_lo(gv[i].z), bf16_lo(xv.z), acc);
-        acc = fmaf(bf16_hi(gv[i].z), bf16_hi(xv.z), acc);
-        acc = fmaf(bf16_lo(gv[i].w), bf16_lo(xv.w), acc);
-        acc = fmaf(bf16_hi(gv[i].w), bf16_hi(xv.w), acc);
-      }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) P.scores[size_t(t) * E + e] = sqrt_softplus_f(acc);
+    for (int i = 0; i < 16; ++i) gv[i] = i < np ? __ldg(grow + lane + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
   }
+  for (int i = threadIdx.x; i < T * H / 8; i += blockDim.x) xs[i] = __ldg(reinterpret_cast<const uint4*>(P.x) + i);
+  if (rank == 0 && P.bias)
+    for (int i = threadIdx.x; i < E; i += blockDim.x) sb[i] = __ldg(P.bias + i);
+  __syncthreads();
+  for (; e < E; e += CL * kRouteWarps) {
+    if (e >= int(rank) * kRouteWarps + kRouteWarps) {  // a further row
+      const uint4* grow = reinterpret_cast<const uint4*>(P.gate + size_t(e) * H);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) gv[i] = i < np ? __ldg(grow + lane + 32 * i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (int t = 0; t < T; ++t) {
+      const uint4* xrow = xs + size_t(t) * (H / 8);
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < np) {
+          const uint4 xv = xrow[lane + 32 * i];
+          acc = fmaf(bf16_lo(gv[i].x), bf16_lo(xv.x), acc);
+          acc = fmaf(bf16_hi(gv[i].x), bf16_hi(xv.x), acc);
+          acc = fmaf(bf16_lo(gv[i].y), bf16_lo(xv.y), acc);
+          acc = fmaf(bf16_hi(gv[i].y), bf16_hi(xv.y), acc);
+          acc = fmaf(bf16_lo(gv[i].z), bf16_lo(xv.z), acc);
+          acc = fmaf(bf16_hi(gv[i].z), bf16_hi(xv.z), acc);
+          acc = fmaf(bf16_lo(gv[i].w), bf16_lo(xv.w), acc);
+          acc = fmaf(bf16_hi(gv[i].w), bf16_hi(xv.w), acc);
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) st_cluster_f32(map_to_rank(sc + size_t(t) * E + e, 0), sqrt_softplus_f(acc));
+    }
+  }
+  cluster_sync_all();  // every score is in the leader's shared memory
+  if (rank != 0) return;
+  // ---- the leader routes the batch
+  if (warp < T) {
+    const float* st = sc + size_t(warp) * E;
+    if (P.token_ids)  // scores in shared memory
+      select_hash_warp<true>(warp, E, P.k, P.vocab, P.routed_scale, st, P.token_ids, P.tid2eid, R.rt.sel_ids,
+                             R.rt.sel_w, P.status);
+    else if (E <= 256)
+      select_compact<8>(warp, E, P.k, P.routed_scale, st, sb, R.rt.sel_ids, R.rt.sel_w);
+    else
+      select_compact<32>(warp, E, P.k, P.routed_scale, st, sb, R.rt.sel_ids, R.rt.sel_w);
+  }
+  __syncthreads();
+  if (warp == 0) route_tables(R.rt, R.tb, P, R.rt.sel_ids, R.rt.sel_w, true);
+  __syncthreads();
+  if (warp == 0) publish_tables(R.tb, P);
+  if (warp == 1)
+    for (int i = lane; i < T * P.k; i += 32) {
+      P.topk_ids[i] = R.rt.sel_ids[i];
+      P.topk_w[i] = R.rt.sel_w[i];
+    }
+  if (warp == 2) write_permutation(R.rt, P, R.tb.nh);
 }
 
 // ---------------------------------------------------------------- w13 kernel
@@ -509,7 +599,6 @@ struct W13Smem {
   float sh_scale[2][kShRows];  // gate / up row scales of this CTA's shared slabs
   Tables tb;
   RouteSmem rt;
-  int ready;          // group 0 has built the tables
 };
 
 constexpr size_t kHead13 = (sizeof(W13Smem) + 127) / 128 * 128;
@@ -620,15 +709,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P, const __gr
   // stages at the next multiple of 1024 bytes (the swizzle's period)
   char* stages = smem + ((smem_u32(smem) + uint32_t(kHead13) + 1023u) & ~1023u) - smem_u32(smem);
   float4* parts = reinterpret_cast<float4*>(stages + size_t(kStages13) * P.stage_bytes);
-  // router scores and bias, outside the ring (it takes the shared slabs
-  // before the routing is known)
-  float* ssc = reinterpret_cast<float*>(reinterpret_cast<char*>(parts) + kPart13);
-  float* sbias = ssc + size_t(P.T) * P.E;
+  // This CTA's intermediates, written to global memory once its slabs are
+  // done (a global store in the slab loop would wait behind the SM's copies
+  // in flight, and so would the fences after it): routed [T][hrs], shared
+  // [T][hss], rows in the order of the CTA's slabs.
+  __half* hst_r = reinterpret_cast<__half*>(reinterpret_cast<char*>(parts) + kPart13);
+  __half* hst_s = hst_r + size_t(P.T) * P.hrs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = P.T, H = P.H;
   const int G = int(gridDim.x), b = int(blockIdx.x);
   const int n_s = P.Is > 0 ? P.Is / 4 : 0;
-  const bool learned = P.layer_mode && !P.token_ids;
+  const int q = warp / kGW, wi = warp % kGW;
+  const int g = lane >> 2, t = lane & 3;
+  const int nkbH = H / 128;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages13; ++s) {
@@ -637,84 +730,68 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P, const __gr
       S.lastfill[s] = -1;
     }
     S.tb.nh = 0;
-    S.ready = 0;
     fence_mbar_init();
   }
   // The w2 kernel may launch now (its CTAs start as these leave their SMs).
   pdl_launch_dependents();
-  // The shared range of this CTA does not depend on the routing: its first
-  // nsp slabs go into the ring before the routing is known.
-  const Chunk c0 = w13_chunk(P, 0, b, G);
-  const int nsp = min(c0.s1 - c0.s0, kStages13);
-  const int q = warp / kGW, wi = warp % kGW;
-  const int g = lane >> 2, t = lane & 3;
-  const int nkbH = H / 128;
 
-  // Global memory outside the ring is read before the first copy is issued:
-  // on this GPU a global load waits behind the SM's transfers in flight. The
-  // loads of the shared slabs' row scales and the bias (into registers,
-  // stored to shared memory after the copies are issued) and of x go out
-  // first.
-  // Group 1 (which takes the shared slabs first) loads the row scales, group
-  // 0 (which selects) the bias, so each group's own barriers order the stores
-  // before its reads.
-  constexpr int kGT = kGW * 32;  // threads per group
-  const int nsr = min(4 * (c0.s1 - c0.s0), kShRows);
-  const int gt = int(threadIdx.x) - q * kGT;  // thread within the group
-  float rsg = 0.f, rsu = 0.f, rb[4] = {0.f, 0.f, 0.f, 0.f};
-  if (q == 1 && gt < nsr) {
-    rsg = __ldg(P.sh13_scale + 4 * c0.s0 + gt);
-    rsu = __ldg(P.sh13_scale + P.Is + 4 * c0.s0 + gt);
-  }
-  if (q == 0 && learned) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (gt + j * kGT < P.E) rb[j] = __ldg(P.bias + gt + j * kGT);
-    for (int i = gt + 4 * kGT; i < P.E; i += kGT) sbias[i] = __ldg(P.bias + i);
-  }
-  // this warp's x slices (token g; in L2 after the router), loaded by each
-  // group when it is about to use them: group 1 at once, group 0 after the
-  // routing, so that the routing code runs with few live registers and no
-  // local-memory traffic (on this GPU that would wait behind the copies in
-  // flight)
+  // Everything this CTA reads from global memory outside the ring is read
+  // before its first copy goes out: on this GPU a load, like an instruction
+  // fetch, waits behind the SM's copies in flight. First what does not
+  // depend on the previous grid: this warp's x slices (token g, K blocks wi
+  // + 8 j; per 32-wide group p the activations kb * 128 + 32 p + 8 t .. + 7,
+  // the MMA steps' K order) and the row scales of the CTA's shared slabs.
   uint32_t B[kNJ][16];
-  auto load_x = [&]() {
-  #pragma unroll
-    for (int j = 0; j < kNJ; ++j) {
-      const int kb = wi + 8 * j;
-      if (kb < nkbH && g < T) {
-        // group p: activations kb * 128 + 32 p + 8 t .. + 7 (the MMA steps' K order)
-        const __nv_bfloat16* src = P.x + size_t(g) * H + kb * 128 + 8 * t;
-  #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + 32 * p));
-          B[j][4 * p] = v.x;
-          B[j][4 * p + 1] = v.y;
-          B[j][4 * p + 2] = v.z;
-          B[j][4 * p + 3] = v.w;
-        }
-      } else {
-  #pragma unroll
-        for (int i = 0; i < 16; ++i) B[j][i] = 0u;
+#pragma unroll
+  for (int j = 0; j < kNJ; ++j) {
+    const int kb = wi + 8 * j;
+    if (kb < nkbH && g < T) {
+      const __nv_bfloat16* src = P.x + size_t(g) * H + kb * 128 + 8 * t;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + 32 * p));
+        B[j][4 * p] = v.x;
+        B[j][4 * p + 1] = v.y;
+        B[j][4 * p + 2] = v.z;
+        B[j][4 * p + 3] = v.w;
       }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) B[j][i] = 0u;
     }
-  };
+  }
+  const Chunk c0 = w13_chunk(P, 0, b, G);  // the shared range does not depend on the routing
+  if (int(threadIdx.x) < min(4 * (c0.s1 - c0.s0), kShRows)) {
+    S.sh_scale[0][threadIdx.x] = __ldg(P.sh13_scale + 4 * c0.s0 + threadIdx.x);
+    S.sh_scale[1][threadIdx.x] = __ldg(P.sh13_scale + P.Is + 4 * c0.s0 + threadIdx.x);
+  }
+  // The shared slabs do not depend on the routing: the first of them go out
+  // now, and have landed by the time the router is done.
+  const int nsp = min(c0.s1 - c0.s0, kStages13);
   __syncthreads();
-  if (warp == 14)
+  if (warp == 0)
     for (int p = 0; p < nsp; ++p)
       fill13(P, M, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, c0.s0 + p), p);
-  if (q == 1 && gt < nsr) {
-    S.sh_scale[0][gt] = rsg;
-    S.sh_scale[1][gt] = rsu;
+  // Then the routing tables: published by the router kernel in layer mode
+  // (complete and visible past the wait), built here from the caller's
+  // routing in forward mode (CTA 0 publishes them for the w2 kernel).
+  pdl_wait();
+  if (P.layer_mode)
+    read_tables(S.tb, P);
+  else if (warp == 0)
+    route_tables(S.rt, S.tb, P, P.topk_ids, P.topk_w, b != 0);
+  __syncthreads();
+  if (!P.layer_mode && b == 0 && warp == 1) publish_tables(S.tb, P);
+  const Chunk ch = w13_chunk(P, S.tb.nh, b, G);
+  const int npos = ch.size();
+  if (warp == 0) {
+    for (int p = nsp; p < kStages13 && p < npos; ++p)
+      fill13(P, M, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, ch.item(p, n_s)), p);
+    if (npos <= kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
   }
-  if (q == 0 && learned) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if (gt + j * kGT < P.E) sbias[gt + j * kGT] = rb[j];
-  }
+
   // ---- f16 activations scaled by 2^sigma (each group keeps its own copy)
-  auto prep_x = [&]() {
-    load_x();
+  {
     uint32_t mx = 0u;
 #pragma unroll
     for (int j = 0; j < kNJ; ++j)
@@ -737,15 +814,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P, const __gr
         B[j][i] = *reinterpret_cast<const uint32_t*>(&hv);
       }
     named_bar_sync(2 + q, kGW * 32);  // the group's sigma is visible to the group
-  };
+  }
 
-  // One slab at ring position pos (chunk ch of npos positions): the warp's K
-  // blocks, its partial tile posted to shared memory; the last warp of the
-  // group to post sums the partials in warp order, refills the stage with
-  // position pos + kStages13 when `refill`, and writes h. False after a
-  // timed-out wait.
-  auto run_item = [&](const Chunk& ch, int npos, int pos, bool refill, bool need_tables) -> bool {
-    const Item m = w13_item(P, S.tb, ch.item(pos, n_s));
+  // One slab at ring position pos: the warp's K blocks, its partial tile
+  // posted to shared memory; the last warp of the group to post sums the
+  // partials in warp order, refills the stage with position pos + kStages13
+  // and stages h. False after a timed-out wait.
+  auto run_item = [&](int pos) -> bool {
+    const int it = ch.item(pos, n_s);
+    const Item m = w13_item(P, S.tb, it);
     const int s = pos % kStages13;
     if (!__all_sync(0xffffffffu, wait_stage(&S.full[s], &S.lastfill[s], pos, kStages13, P))) return false;
     const char* st = stages + size_t(s) * P.stage_bytes;
@@ -783,40 +860,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P, const __gr
     }
     if (lane == 0) S.redcnt[s] = 0;
     __syncwarp();
-    if (refill) {
-      Chunk cr = ch;
-      int nr = npos;
-      bool have = true;
-      if (need_tables) {  // the next position may be routed: wait for the tables
-        uint32_t i = 0;
-        while (*reinterpret_cast<volatile int*>(&S.ready) == 0 && ++i < kBarTries) __nanosleep(32);
-        have = i < kBarTries;
-        if (!have && lane == 0) atomicOr(P.status, kStatusTimeout);
-        __threadfence_block();
-        cr = w13_chunk(P, S.tb.nh, b, G);
-        nr = cr.size();
-      }
-      if (have && pos + kStages13 < nr) {
-        fill13(P, M, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, cr.item(pos + kStages13, n_s)),
-               pos + kStages13);
-        if (pos + kStages13 == nr - 1 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
-      }
-      if (!have) return false;
+    if (pos + kStages13 < npos) {
+      fill13(P, M, S, stages + size_t(s) * P.stage_bytes, s, w13_item(P, S.tb, ch.item(pos + kStages13, n_s)),
+             pos + kStages13);
+      if (pos + kStages13 == npos - 1 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
     }
     const float dg[2] = {d.x, d.y}, du[2] = {d.z, d.w};
     if (m.kind == kR13) {
-      const uint32_t mask = S.tb.mask[m.li];
+      const int rl = (it - n_s - ch.r0) * 8 + g;  // row among this CTA's routed rows
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
         const int tok = 2 * t + qq;
-        if (tok < T && ((mask >> tok) & 1u)) {
+        if (tok < T) {
           const float inv = pow2f(-S.sigma[q][tok]);
           const float h = clamped_swiglu_f(dg[qq] * inv, du[qq] * inv, P.limit) * S.tb.w[m.li * 8 + tok] * P.tau_r;
-          P.dh[(size_t(m.li) * T + tok) * P.I + m.row0 + g] = __float2half_rn(h);
+          hst_r[tok * P.hrs + rl] = __float2half_rn(h);
         }
       }
     } else if (g < 4) {
-      const int rl = m.row0 + g - 4 * ch.s0;  // row within this CTA's shared slabs
+      const int rl = m.row0 + g - 4 * ch.s0;  // row among this CTA's shared rows
       const float sg = rl < kShRows ? S.sh_scale[0][rl] : __ldg(P.sh13_scale + m.row0 + g);
       const float su = rl < kShRows ? S.sh_scale[1][rl] : __ldg(P.sh13_scale + P.Is + m.row0 + g);
 #pragma unroll
@@ -824,7 +886,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P, const __gr
         const int tok = 2 * t + qq;
         if (tok < T) {
           const float inv = pow2f(-S.sigma[q][tok]);
-          P.hs[size_t(tok) * P.Is + m.row0 + g] =
+          hst_s[tok * P.hss + rl] =
               __float2half_rn(clamped_swiglu_f(dg[qq] * sg * inv, du[qq] * su * inv, P.limit) * P.tau_s);
         }
       }
@@ -832,69 +894,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w13(DecParams P, const __gr
     return true;
   };
 
+  // ---- item loop: group q takes ring positions q, q + 2, ... (shared slabs
+  // first, then routed)
   bool ok = true;
-  if (q == 1) {
-    // ---- group 1: the shared slabs already on their way, while group 0
-    // routes; their refills continue with the following positions
-    prep_x();
-    for (int pos = 0; pos < nsp && ok; ++pos) ok = run_item(c0, nsp, pos, true, true);
-  } else {
-    // ---- group 0: routing. Every CTA selects from the scores and builds the
-    // tables; the scores (previous grid) are complete and visible past the wait.
-    pdl_wait();
-    if (P.layer_mode) {
-      for (int i = threadIdx.x; i < T * P.E; i += kGT) ssc[i] = __ldcg(P.scores + i);
-      named_bar_sync(4, kGT);
-      if (warp < T) select_token(S.rt, P, warp, ssc, sbias);
-      named_bar_sync(4, kGT);
-      if (warp == 0) route_tables(S.rt, S.tb, P, S.rt.sel_ids, S.rt.sel_w, true);
-    } else if (warp == 0) {
-      route_tables(S.rt, S.tb, P, P.topk_ids, P.topk_w, b != 0);
-    }
-    named_bar_sync(4, kGT);
-    if (warp == 0) {
-      // the stages the shared slabs did not take, then the tables are ready
-      // for group 1's refills
-      const Chunk cr = w13_chunk(P, S.tb.nh, b, G);
-      const int nr = cr.size();
-      for (int p = nsp; p < kStages13 && p < nr; ++p)
-        fill13(P, M, S, stages + size_t(p) * P.stage_bytes, p, w13_item(P, S.tb, cr.item(p, n_s)), p);
-      if (nr <= kStages13 && lane == 0) prefetch_w2_share(P, S.tb, b, true);
-      __threadfence_block();
-      if (lane == 0) *reinterpret_cast<volatile int*>(&S.ready) = 1;
-    }
-    if (b == 0) {  // one CTA writes the routing outputs and the w2 kernel's tables
-      if (warp == 1) publish_tables(S.tb, P);
-      if (P.layer_mode && warp == 2)
-        for (int i = lane; i < T * P.k; i += 32) {
-          P.topk_ids[i] = S.rt.sel_ids[i];
-          P.topk_w[i] = S.rt.sel_w[i];
-        }
-      if (P.layer_mode && warp == 3) write_permutation(S.rt, P, S.tb.nh);
-    }
-    prep_x();
-  }
-  if (q == 1) {
-    // group 0's tables, before this group's first routed position
-    uint32_t i = 0;
-    while (*reinterpret_cast<volatile int*>(&S.ready) == 0 && ++i < kBarTries) __nanosleep(32);
-    if (i >= kBarTries) {
-      ok = false;
-      if (lane == 0) atomicOr(P.status, kStatusTimeout);
-    }
-    __threadfence_block();
-  }
-  const Chunk ch = w13_chunk(P, S.tb.nh, b, G);
-  const int npos = ch.size();
-
-  // ---- item loop: group q takes ring positions nsp + q, nsp + q + 2, ...
-  for (int pos = nsp + q; pos < npos && ok; pos += 2) ok = run_item(ch, npos, pos, true, false);
+  for (int pos = q; pos < npos && ok; pos += 2) ok = run_item(pos);
   // No copy may still be landing in this CTA's shared memory (possible only
   // after a timeout).
   __syncthreads();
   if (threadIdx.x == 0)
     for (int s = 0; s < kStages13; ++s)
       if (S.lastfill[s] >= 0) mbar_wait_bounded(&S.full[s], uint32_t(S.lastfill[s] / kStages13) & 1u, kBarTries);
+  // The staged intermediates: routed rows of the tokens routed to the
+  // expert (the w2 kernel reads no others), every shared row.
+  const int nrr = (ch.r1 - ch.r0) * 8, nsr2 = (ch.s1 - ch.s0) * 4;
+  for (int i = threadIdx.x; i < T * nrr; i += blockDim.x) {
+    const int tok = i / nrr, f = ch.r0 * 8 + i % nrr;  // row of the flattened [nh, I] list
+    const int li = f / P.I;
+    if ((S.tb.mask[li] >> tok) & 1u) P.dh[(size_t(li) * T + tok) * P.I + f % P.I] = hst_r[tok * P.hrs + i % nrr];
+  }
+  for (int i = threadIdx.x; i < T * nsr2; i += blockDim.x) {
+    const int tok = i / nsr2, r = i % nsr2;
+    P.hs[size_t(tok) * P.Is + ch.s0 * 4 + r] = hst_s[tok * P.hss + r];
+  }
 }
 
 // ---------------------------------------------------------------- w2 kernel
@@ -1125,12 +1146,50 @@ float h_scale(float bound) {
 }
 
 struct Plan {
-  int stage13 = 0, stage2 = 0, nst2 = 0;
+  int stage13 = 0, stage2 = 0, nst2 = 0, hrs = 0, hss = 0;
   size_t smem13 = 0, smem2 = 0;
   bool ok = false;
 };
 
-Plan make_plan(const v4moe_config& c, int T) {
+size_t route_smem_bytes(const v4moe_config& c, int T) {
+  return kRouteTail + (size_t(T) * c.n_experts + c.n_experts) * 4 + 16 + size_t(T) * c.hidden * 2;
+}
+
+// Router cluster size: the largest of 16, 8, 4, 2 CTAs (at most one per 16
+// experts' warps) that the device can co-schedule with this shared memory;
+// queried once per device and size class. 0 if none.
+int route_cluster(size_t smem) {
+  static std::mutex mu;
+  static std::map<std::pair<int, size_t>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(dev, smem);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  cudaFuncSetAttribute(k_dec_route, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  int best = 0;
+  for (int cl = kRouteMaxCluster; cl >= 2 && best == 0; cl /= 2) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cl);
+    cfg.blockDim = dim3(kRouteWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(cl);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_dec_route, &cfg) == cudaSuccess && n >= 1) best = cl;
+  }
+  cudaGetLastError();  // a refused size leaves no sticky error
+  cache[key] = best;
+  return best;
+}
+
+Plan make_plan(const v4moe_config& c, int T, int G) {
   Plan p;
   if (T < 1 || T > kDecodeMaxTokens || T * c.top_k > kMaxHit) return p;
   const int H = c.hidden, I = c.inter, Is = c.shared_inter;
@@ -1141,14 +1200,19 @@ Plan make_plan(const v4moe_config& c, int T) {
   if (H % 512 != 0 || I % 512 != 0 || !pow2(H) || !pow2(I) || Is % 128 != 0) return p;
   const int s13 = std::max(8 * H + 2 * align1k(8 * (H / 32)), Is > 0 ? 8 * H : 0);
   p.stage13 = align1k(s13);
-  const size_t route_stage = (size_t(T) * c.n_experts + c.n_experts) * 4;  // scores + bias
+  // staged intermediates: a CTA's share of the routed rows (at most
+  // min(E, T k) experts hit) and of the shared rows, per token
+  const int nh_max = std::min(c.n_experts, T * c.top_k);
+  p.hrs = (nh_max * (I / 8) + G - 1) / G * 8;
+  p.hss = (Is / 4 + G - 1) / G * 4;
+  const size_t hstage = size_t(T) * (p.hrs + p.hss) * 2;
   // 1024 bytes of slack put the first stage on a multiple of 1024
-  p.smem13 = kHead13 + 1024 + size_t(kStages13) * p.stage13 + kPart13 + (route_stage + 127) / 128 * 128;
+  p.smem13 = kHead13 + 1024 + size_t(kStages13) * p.stage13 + kPart13 + (hstage + 127) / 128 * 128;
   p.stage2 = align1k(w2_hoff(I, Is) + T * std::max(I, Is) * 2);
   const size_t room = 227 * 1024 - kHead2 - 1024 - kRed2;
   p.nst2 = int(std::min<size_t>(kMaxStages2, room / p.stage2));
   p.smem2 = kHead2 + 1024 + size_t(p.nst2) * p.stage2 + kRed2;
-  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 && size_t(T) * H * 2 <= 227 * 1024;
+  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 && route_smem_bytes(c, T) <= 227 * 1024;
   return p;
 }
 
@@ -1193,15 +1257,15 @@ DecodeBuffers dec_buffers(const v4moe_config& c, int64_t T) {
   return b;
 }
 
-bool dec_supported(const v4moe_config& c, int T) { return make_plan(c, T).ok; }
+bool dec_supported(const v4moe_config& c, int T) { return make_plan(c, T, device_sms()).ok; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const v4moe_config& c = a.c;
-  const Plan p = make_plan(c, a.T);
+  const int sms = device_sms();
+  const Plan p = make_plan(c, a.T, sms);
   if (!p.ok) return cudaErrorInvalidValue;
   DecMaps m13, m2;
   if (!dec_maps(c, a.w, m13, m2)) return cudaErrorInvalidValue;
-  const int sms = device_sms();
   DecParams P;
   P.T = a.T;
   P.H = c.hidden;
@@ -1222,6 +1286,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   P.stage_bytes = 0;
   P.nstages = 0;
   P.w2_per = 1;
+  P.hrs = p.hrs;
+  P.hss = p.hss;
   P.x = a.x;
   P.gate = a.gate;
   P.bias = a.bias;
@@ -1253,10 +1319,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   const int grid2 = (nrb + P.w2_per - 1) / P.w2_per;
   cudaError_t e = cudaSuccess;
   if (a.layer_mode) {
-    const size_t route_smem = size_t(a.T) * c.hidden * 2;
+    const size_t route_smem = route_smem_bytes(c, a.T);
     set_smem(k_dec_route, route_smem);
-    e = launch_kernel("dec_route", k_dec_route, dim3((c.n_experts + kRouteWarps - 1) / kRouteWarps),
-                      dim3(kRouteWarps * 32), route_smem, st, false, P);
+    const int cl = route_cluster(route_smem);
+    if (cl <= 0) return cudaErrorInvalidValue;
+    e = launch_kernel_cl("dec_route", k_dec_route, dim3(cl), dim3(kRouteWarps * 32), route_smem, st, false, cl, P);
     if (e != cudaSuccess) return e;
   }
   // Without a routing kernel in front, the w13 kernel must not overlap the

@@ -77,12 +77,12 @@ def test_swiglu_clamp_engaged(name, T, H, E, I, Is):
     run_parity(li, _layer(li))
 
 
-def _tie_inputs(T, E, H=512, seed=3):
+def _tie_inputs(T, E, H=512, seed=3, I=256):
     """Gate rows one-hot (value 1) so that z_e = x[t, col(e)] exactly; experts 4
     and 8 read the same column, so their scores (and, with a zero bias, their
     biased scores) tie exactly in fp32 and in fp64. Every token has five
     clear winners above that pair and everything else below it."""
-    wl = IN.Workload("ties", T=T, H=H, E=E, I=256, Is=256, bias_std=0.0, seed=seed)
+    wl = IN.Workload("ties", T=T, H=H, E=E, I=I, Is=256, bias_std=0.0, seed=seed)
     li = IN.make_layer_inputs(wl)
     col = np.arange(E)
     col[8] = 4
@@ -105,12 +105,15 @@ def _tie_inputs(T, E, H=512, seed=3):
     return _with(li, gate=gate, x=x, bias=np.zeros(E, np.float32))
 
 
-@pytest.mark.parametrize("T,E", [(5, 16), (40, 16), (3, 300)])
-def test_exact_tie_goes_to_lower_expert_id(T, E):
+# I = 512 puts batches of at most 8 tokens on the decode kernels, whose router
+# selects inside the whole-layer call (E = 300: more experts than its warps,
+# and more than 256 per token)
+@pytest.mark.parametrize("T,E,I", [(5, 16, 256), (40, 16, 256), (3, 300, 256), (5, 16, 512), (3, 300, 512)])
+def test_exact_tie_goes_to_lower_expert_id(T, E, I):
     """An exact tie at the 6th place: the lower id (4) is chosen on the GPU,
     by the standalone router and inside the whole-layer call, on every
     token (no near-tie exclusion here)."""
-    li = _tie_inputs(T, E)
+    li = _tie_inputs(T, E, I=I)
     lay = O.Layer(li)
     ids_o, w_o, margin, _ = lay.route()
     assert (margin == 0.0).all()

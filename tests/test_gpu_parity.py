@@ -59,6 +59,24 @@ def test_hash_routing_small(T):
     run_parity(li, _layer(li))
 
 
+@pytest.mark.parametrize("T", [1, 5, 8])
+def test_decode_hash_routing(T):
+    """Hash routing on the decode kernels (at most 8 tokens, K a power of two
+    from 512): the router's leader reads the token ids and the table."""
+    wl = IN.Workload("dec_hash", T=T, H=1024, E=32, I=512, Is=256, routing="hash", vocab=1000, seed=23)
+    li = IN.make_layer_inputs(wl)
+    run_parity(li, _layer(li))
+
+
+@pytest.mark.parametrize("T", [2, 8])
+def test_decode_more_experts_than_router_warps(T):
+    """E = 320: the decode router's warps score a second row each, and the
+    selection holds 10 scores per lane."""
+    wl = IN.Workload("dec_e320", T=T, H=1024, E=320, I=512, Is=256, bias_std=0.05, seed=29)
+    li = IN.make_layer_inputs(wl)
+    run_parity(li, _layer(li))
+
+
 @pytest.mark.parametrize("T", [3, 50])
 def test_no_shared_expert_and_k1(T):
     wl = IN.Workload("noshared", T=T, H=256, E=8, k=1, I=128, Is=0, seed=2)
