@@ -31,11 +31,12 @@
 //    in warp order, refills the stage and stages h as f16 (routed: w * h) in
 //    shared memory; the CTA writes its h rows once its slabs are done.
 //  * k_dec_w2: two groups of eight warps, warp i of a group owning K blocks
-//    i, i + 8. CTA b owns a run of 16-row output blocks and goes through the
-//    shared expert and every routed expert for each of them, the two groups
-//    taking alternate experts; a stage holds
-//    the expert's 16 weight rows and the intermediates of its tokens. The sum
-//    over experts (shared first, then ascending id) is formed in registers and
+//    i, i + 8. CTA b owns a run of (at most two) 16-row output blocks; its
+//    ring positions are the blocks' (expert, block) items, the shared expert
+//    first, then the routed experts in ascending id, and group q takes the
+//    positions q, q + 2, ...; a stage holds the expert's 16 weight rows and
+//    the intermediates of its tokens. Each warp sums its items per block in
+//    registers; at the end the sixteen warps' sums are added in warp order and
 //    written once as bf16, so the result does not depend on timing.
 //
 // The intermediates are stored as f16 scaled by a fixed power of two chosen
@@ -928,7 +929,8 @@ struct W2Smem {
   Tables tb;
 };
 constexpr size_t kHead2 = (sizeof(W2Smem) + 127) / 128 * 128;
-constexpr size_t kRed2 = size_t(16) * 32 * 16;  // float4 per lane and warp
+constexpr int kW2Blocks = 2;  // 16-row output blocks per w2 CTA, at most
+constexpr size_t kRed2 = size_t(kW2Blocks) * 16 * 32 * 16;  // float4 per lane, warp and block
 
 // Ring position p of CTA b: output block rb = b w2_per + p / nl, expert slot
 // l = p % nl (the shared expert first when there is one, then the routed list).
@@ -1033,101 +1035,106 @@ __global__ void __launch_bounds__(kThreads, 1) k_dec_w2(DecParams P, const __gri
     mbar_arrive(&S.full[0]);
   }
 
-  // Two groups of eight warps take alternate expert slots of each output
-  // block; warp i of a group owns K blocks i, i + 8. Every warp keeps its
-  // partial sums over the block's experts in registers; at the end of the
-  // block all sixteen are summed in warp order.
+  // Two groups of eight warps take alternate ring positions (group q the
+  // positions q, q + 2, ... of the CTA's blocks x experts); warp i of a group
+  // owns K blocks i, i + 8. Every warp keeps its partial sums per output
+  // block in registers; once all positions are done the sixteen warps'
+  // partials of each block are summed in warp order.
   const int q = warp >> 3, wi = warp & 7;
   bool ok = true;
-  for (int r = 0; r < nrb_mine; ++r) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int l = q; l < nl; l += 2) {
-      const int pos = r * nl + l;
-      const Item2 m = w2_item(P, nl, b, pos);
-      const int s = pos % NS;
-      // A timed-out warp keeps going (without reading the stage) so that every
-      // warp reaches the block-end barriers.
-      ok = ok && __all_sync(0xffffffffu, wait_stage(&S.full[s], &S.lastfill[s], pos, NS, P));
-      if (!ok) continue;
-      const char* st = stages + size_t(s) * P.stage_bytes;
-      const bool sh = m.li < 0;
-      const int K = sh ? P.Is : P.I;
-      const int nkb = K / 128;
-      // B: the intermediates of token g (zero for tokens not routed here)
-      const uint32_t mask = sh ? (1u << T) - 1u : S.tb.mask[m.li];
-      const bool has_tok = g < T && ((mask >> g) & 1u);
-      uint32_t Bf[2][16];
+  float4 acc[kW2Blocks];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int kb = wi + 8 * j;
-        if (has_tok && kb < nkb) {
-          load_b_smem(st + w2_hoff(P.I, P.Is) + g * K * 2, kb, Bf[j]);
-        } else {
+  for (int i = 0; i < kW2Blocks; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int pos = q; pos < n_items; pos += 2) {
+    const Item2 m = w2_item(P, nl, b, pos);
+    const int s = pos % NS;
+    // A timed-out warp keeps going (without reading the stage) so that every
+    // warp reaches the final barriers.
+    ok = ok && __all_sync(0xffffffffu, wait_stage(&S.full[s], &S.lastfill[s], pos, NS, P));
+    if (!ok) continue;
+    const char* st = stages + size_t(s) * P.stage_bytes;
+    const bool sh = m.li < 0;
+    const int K = sh ? P.Is : P.I;
+    const int nkb = K / 128;
+    const int rr = m.rb - b * P.w2_per;  // block within this CTA's
+    // B: the intermediates of token g (zero for tokens not routed here)
+    const uint32_t mask = sh ? (1u << T) - 1u : S.tb.mask[m.li];
+    const bool has_tok = g < T && ((mask >> g) & 1u);
+    uint32_t Bf[2][16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) Bf[j][i] = 0u;
-        }
-      }
-      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-      if (sh) {
-        tile_s8<2, 8>(st, g, st, g + 8, 16, true, wi, nkb, Bf, a0, a1);
-        const int rl = (m.rb - b * P.w2_per) * 16 + g;  // row within this CTA's output rows
-        const float its = 1.0f / P.tau_s;
-        const float sa = (rl < kShRows ? S.sh_scale[rl] : __ldg(P.sh2_scale + m.rb * 16 + g)) * its;
-        const float sb = (rl + 8 < kShRows ? S.sh_scale[rl + 8] : __ldg(P.sh2_scale + m.rb * 16 + g + 8)) * its;
-        acc.x += (a0[0] + a1[0]) * sa;
-        acc.y += (a0[1] + a1[1]) * sa;
-        acc.z += (a0[2] + a1[2]) * sb;
-        acc.w += (a0[3] + a1[3]) * sb;
+    for (int j = 0; j < 2; ++j) {
+      const int kb = wi + 8 * j;
+      if (has_tok && kb < nkb) {
+        load_b_smem(st + w2_hoff(P.I, P.Is) + g * K * 2, kb, Bf[j]);
       } else {
-        const char* sc = st + 8 * P.I;  // the scale box after the 16-row code box
-        tile_mx<2, 8>(st, g, st, g + 8, 16, sc, sc, P.I / 32, wi, nkb, Bf, a0);
-        const float itr = 1.0f / P.tau_r;
-        acc.x += a0[0] * itr;
-        acc.y += a0[1] * itr;
-        acc.z += a0[2] * itr;
-        acc.w += a0[3] * itr;
-      }
-      // the last warp of the group to finish with the stage refills it
-      __syncwarp();
-      int old = 0;
-      if (lane == 0) old = atomicAdd(&S.redcnt[s], 1);
-      old = __shfl_sync(0xffffffffu, old, 0);
-      if (old == 7) {
-        if (lane == 0) S.redcnt[s] = 0;
-        __syncwarp();
-        const int np = pos + NS;
-        if (np < n_items) {
-          const Item2 mn = w2_item(P, nl, b, np);
-          if (lane == 0) {
-            S.lastfill[s] = np;
-            fill2_weights(P, M, S, stages + size_t(s) * P.stage_bytes, s, mn);
-          }
-          __syncwarp();
-          fill2_h(P, S, stages + size_t(s) * P.stage_bytes, s, mn);
-        }
-      }
-    }
-    // block done: sum the 16 warps' partials in warp order, write bf16
-    red[warp * 32 + lane] = acc;
-    __syncthreads();
-    if (warp == 0) {
-      float4 d = red[lane];
-      for (int w = 1; w < 16; ++w) {
-        const float4 v = red[w * 32 + lane];
-        d.x += v.x;
-        d.y += v.y;
-        d.z += v.z;
-        d.w += v.w;
-      }
-      const float v[4] = {d.x, d.y, d.z, d.w};
-      const int rb = b * P.w2_per + r;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int tok = 2 * t + (i & 1);
-        if (tok < T) P.out[size_t(tok) * P.H + rb * 16 + g + 8 * (i >> 1)] = __float2bfloat16_rn(v[i]);
+        for (int i = 0; i < 16; ++i) Bf[j][i] = 0u;
       }
     }
-    __syncthreads();
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 d;
+    if (sh) {
+      tile_s8<2, 8>(st, g, st, g + 8, 16, true, wi, nkb, Bf, a0, a1);
+      const int rl = rr * 16 + g;  // row within this CTA's output rows
+      const float its = 1.0f / P.tau_s;
+      const float sa = (rl < kShRows ? S.sh_scale[rl] : __ldg(P.sh2_scale + m.rb * 16 + g)) * its;
+      const float sb = (rl + 8 < kShRows ? S.sh_scale[rl + 8] : __ldg(P.sh2_scale + m.rb * 16 + g + 8)) * its;
+      d = make_float4((a0[0] + a1[0]) * sa, (a0[1] + a1[1]) * sa, (a0[2] + a1[2]) * sb, (a0[3] + a1[3]) * sb);
+    } else {
+      const char* sc = st + 8 * P.I;  // the scale box after the 16-row code box
+      tile_mx<2, 8>(st, g, st, g + 8, 16, sc, sc, P.I / 32, wi, nkb, Bf, a0);
+      const float itr = 1.0f / P.tau_r;
+      d = make_float4(a0[0] * itr, a0[1] * itr, a0[2] * itr, a0[3] * itr);
+    }
+#pragma unroll
+    for (int i = 0; i < kW2Blocks; ++i)
+      if (i == rr) {
+        acc[i].x += d.x;
+        acc[i].y += d.y;
+        acc[i].z += d.z;
+        acc[i].w += d.w;
+      }
+    // the last warp of the group to finish with the stage refills it
+    __syncwarp();
+    int old = 0;
+    if (lane == 0) old = atomicAdd(&S.redcnt[s], 1);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    if (old == 7) {
+      if (lane == 0) S.redcnt[s] = 0;
+      __syncwarp();
+      const int np = pos + NS;
+      if (np < n_items) {
+        const Item2 mn = w2_item(P, nl, b, np);
+        if (lane == 0) {
+          S.lastfill[s] = np;
+          fill2_weights(P, M, S, stages + size_t(s) * P.stage_bytes, s, mn);
+        }
+        __syncwarp();
+        fill2_h(P, S, stages + size_t(s) * P.stage_bytes, s, mn);
+      }
+    }
+  }
+  // every block: the sixteen warps' partials summed in warp order, bf16
+#pragma unroll
+  for (int i = 0; i < kW2Blocks; ++i) red[(i * 16 + warp) * 32 + lane] = acc[i];
+  __syncthreads();
+  if (warp < nrb_mine) {
+    const int r = warp;
+    float4 d = red[(r * 16) * 32 + lane];
+    for (int w = 1; w < 16; ++w) {
+      const float4 v = red[(r * 16 + w) * 32 + lane];
+      d.x += v.x;
+      d.y += v.y;
+      d.z += v.z;
+      d.w += v.w;
+    }
+    const float v[4] = {d.x, d.y, d.z, d.w};
+    const int rb = b * P.w2_per + r;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tok = 2 * t + (i & 1);
+      if (tok < T) P.out[size_t(tok) * P.H + rb * 16 + g + 8 * (i >> 1)] = __float2bfloat16_rn(v[i]);
+    }
   }
   // No copy may still be landing in this CTA's shared memory.
   __syncthreads();
@@ -1212,7 +1219,8 @@ Plan make_plan(const v4moe_config& c, int T, int G) {
   const size_t room = 227 * 1024 - kHead2 - 1024 - kRed2;
   p.nst2 = int(std::min<size_t>(kMaxStages2, room / p.stage2));
   p.smem2 = kHead2 + 1024 + size_t(p.nst2) * p.stage2 + kRed2;
-  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 && route_smem_bytes(c, T) <= 227 * 1024;
+  p.ok = p.smem13 <= 227 * 1024 && p.nst2 >= 2 && route_smem_bytes(c, T) <= 227 * 1024 &&
+         (H / 16 + G - 1) / G <= kW2Blocks;
   return p;
 }
 
