@@ -189,7 +189,7 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t w) {
 
 // Whole CTA; the caller synchronises afterwards.
 __device__ __forceinline__ void read_tables(Tables& tb, const DecParams& P) {
-  const int nh = int(__ldcg(P.ctl + cNh));
+  const int nh = min(max(int(__ldcg(P.ctl + cNh)), 0), kMaxHit);  // bounded whatever the word holds
   for (int i = threadIdx.x; i < nh; i += blockDim.x) {
     tb.hit[i] = int(__ldcg(P.ctl + cHit + i));
     tb.mask[i] = __ldcg(P.ctl + cMask + i);
