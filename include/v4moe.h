@@ -186,10 +186,13 @@ int32_t v4moe_forward(const v4moe_config* cfg, int32_t T, const void* x,
 
 /* The whole layer in one call: v4moe_route, v4moe_permute and v4moe_forward
  * with the same arguments and results (routing outputs included). For small
- * batches (T <= 8) the router scores run in one small kernel and the expert
- * kernels, chained to it by programmatic dependent launch, select each
- * token's experts themselves while they already stream the shared expert's
- * weights. */
+ * batches (T <= 8) the router runs as one thread-block cluster (up to 16
+ * CTAs) whose leader selects each token's experts and writes the routing
+ * outputs and the permutation, and the two expert kernels, chained to it by
+ * programmatic dependent launch, start streaming the shared expert's weights
+ * before the routing is known. Intermediates on this path are f16 of h
+ * times a fixed power of two derived from swiglu_limit (divided out in the
+ * down projection). */
 int32_t v4moe_layer(const v4moe_config* cfg, int32_t T, const void* x, const void* gate,
                     const float* bias, const int32_t* token_ids, const int32_t* tid2eid,
                     const v4moe_weights* weights, int32_t* topk_ids, float* topk_w,
