@@ -25,10 +25,10 @@ backend; the tests use two gloo ranks on the CPU):
 The fused device form (dispatch written by the router's permutation kernel
 straight into the owner's receive buffer, combine written by the down
 projection's epilogue into the home rank's slot rows, over NVLink peer
-stores with a flag per source rank) keeps these orders; it is not built here
-(one GPU per process in this environment). Remote rows are stored into the
-receiving GPU's own memory before any kernel reads them: no tensor-memory
-copy with cluster multicast and no library GEMM is given another GPU's memory.
+stores with a flag per source rank) keeps these orders; the library does not
+contain it yet. Remote rows are to be stored into the receiving GPU's own
+memory before any kernel reads them: no tensor-memory copy with cluster
+multicast and no library GEMM is given another GPU's memory.
 """
 from __future__ import annotations
 
