@@ -12,7 +12,8 @@
 //     out_t = W2_shared hs_t + sum over the token's experts of w * W2_e h.
 //
 // Kernels:
-//  * k_dec_route: router scores (one warp per expert); the last CTA to finish
+//  * k_dec_route: one thread-block cluster; each warp scores experts into the
+//    leader CTA's shared memory, and after the cluster barrier the leader
 //    selects each token's experts and publishes the batch's routing tables
 //    (distinct experts in ascending id, token masks, weights), the routing
 //    outputs and the permutation.
@@ -114,7 +115,6 @@ struct DecParams {
   int32_t* offsets;
   int32_t* sorted_slot;
   int32_t* slot_pos;
-  float* scores;  // [T, E]
   const uint8_t* w13_codes;
   const uint8_t* w13_scales;
   const uint8_t* w2_codes;
@@ -1307,7 +1307,6 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
   P.offsets = a.offsets;
   P.sorted_slot = a.sorted_slot;
   P.slot_pos = a.slot_pos;
-  P.scores = a.scores;
   P.w13_codes = a.w.w13_codes;
   P.w13_scales = a.w.w13_scales;
   P.w2_codes = a.w.w2_codes;

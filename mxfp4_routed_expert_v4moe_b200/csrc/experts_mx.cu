@@ -36,7 +36,6 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "launch.cuh"
 #include "ptx.cuh"
@@ -940,23 +939,10 @@ __global__ void __launch_bounds__(kXThreads, 1)
 }
 
 
-PFN_cuTensorMapEncodeTiled_v12000 mx_encode_fn() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // 3-D map of the w13 codes: {K, I rows of a half, 2 E halves}; box {128, 64, 2}
 // brings a tile's 64 gate rows and the matching 64 up rows in one copy.
 bool mx_map_w13(CUtensorMap* m, const void* base, uint64_t K, uint64_t I, uint64_t halves) {
-  auto fn = mx_encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t dims[3] = {K, I, halves};
   const cuuint64_t strides[2] = {K / 2, I * (K / 2)};
@@ -970,7 +956,7 @@ bool mx_map_w13(CUtensorMap* m, const void* base, uint64_t K, uint64_t I, uint64
 // 2-D map, 128-byte swizzle, box {128 elements, box_rows}.
 bool mx_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t row_bytes, uint64_t rows,
             uint32_t box_rows) {
-  auto fn = mx_encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   if (rows == 0) rows = 1;
   const cuuint64_t dims[2] = {cols, rows};
@@ -985,7 +971,7 @@ bool mx_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t c
 // General 2-D / 3-D maps ([halves][rows][cols], rows row_bytes apart).
 bool mx_map2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t row_bytes, uint64_t rows,
               uint32_t bx, uint32_t by, CUtensorMapSwizzle sw) {
-  auto fn = mx_encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   if (rows == 0) rows = 1;
   const cuuint64_t dims[2] = {cols, rows};
@@ -998,7 +984,7 @@ bool mx_map2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t
 
 bool mx_map3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t row_bytes, uint64_t rows,
               uint64_t halves, uint32_t bx, uint32_t by, CUtensorMapSwizzle sw) {
-  auto fn = mx_encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t dims[3] = {cols, rows, halves};
   const cuuint64_t strides[2] = {row_bytes, rows * row_bytes};
@@ -1014,7 +1000,7 @@ bool mx_supported(const v4moe_config& c, const v4moe_weights& w) {
   auto a32 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; };
   return c.hidden % 512 == 0 && c.inter % 512 == 0 && a32(w.w13_codes) && a32(w.w2_codes) &&
          (reinterpret_cast<uintptr_t>(w.w13_scales) & 15) == 0 && (reinterpret_cast<uintptr_t>(w.w2_scales) & 15) == 0 &&
-         mx_encode_fn() != nullptr;
+         tensor_map_encoder() != nullptr;
 }
 
 cudaError_t launch_mx_gather(const ForwardArgs& a, __half* x16, int* sigma, const MxBuffers& m, cudaStream_t st) {

@@ -33,7 +33,6 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "launch.cuh"
 #include "ptx.cuh"
@@ -608,23 +607,10 @@ __global__ void __launch_bounds__(1024) k_tc_tiles(int T, int E, int H, int I, i
 
 // ------------------------------------------------------------------ host
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // 2-D map over a row-major [rows, cols] tensor; box {box_cols, box_rows}.
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols, uint64_t rows,
               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   if (rows == 0) rows = 1;
   const cuuint64_t dims[2] = {cols, rows};

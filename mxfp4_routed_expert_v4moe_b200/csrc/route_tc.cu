@@ -16,7 +16,6 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "launch.cuh"
 #include "ptx.cuh"
@@ -193,22 +192,9 @@ __global__ void __launch_bounds__(256) k_route_select(int T, int E, int k, int k
     select_learned<false>(t, E, k, routed_scale, s, bias, topk_ids, topk_w);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 rt_encode_fn() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // bf16 [rows, cols] row-major, 128-byte swizzle, box {64, box_rows}.
 bool rt_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
-  auto fn = rt_encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};

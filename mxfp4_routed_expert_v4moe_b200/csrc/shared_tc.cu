@@ -36,7 +36,6 @@
 
 #include <algorithm>
 #include <cmath>
-#include <mutex>
 
 #include "launch.cuh"
 #include "ptx.cuh"
@@ -458,24 +457,11 @@ __global__ void __launch_bounds__(256) k_s8_to_bf16(const int8_t* __restrict__ q
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 sh_encode_fn() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // 16-bit maps (f16 unless given), 128-byte swizzle, box of 64 elements (128 B)
 // along K. 2-D: [rows][cols]; 3-D: [2][rows][cols] (gate half, up half).
 bool sh_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t halves, uint32_t box_rows,
             CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT16) {
-  auto fn = sh_encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   if (rows == 0) rows = 1;
   const cuuint64_t dims[3] = {cols, rows, halves};
@@ -491,7 +477,7 @@ bool sh_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint
 
 bool sh_supported(const v4moe_config& c, int64_t T) {
   return c.shared_inter > 0 && T >= kShMinTokens && c.shared_inter % 128 == 0 && c.hidden % 256 == 0 &&
-         sh_encode_fn() != nullptr;
+         tensor_map_encoder() != nullptr;
 }
 
 size_t sh_extra_bytes(const v4moe_config& c, int64_t T) {

@@ -65,8 +65,7 @@ int device_sms() {
   return d && d->sms > 0 ? d->sms : 148;
 }
 
-bool encode_tensor_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-                       const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   std::call_once(once, [] {
@@ -76,6 +75,12 @@ bool encode_tensor_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const v
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
+  return fn;
+}
+
+bool encode_tensor_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                       const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
+  const auto fn = tensor_map_encoder();
   if (!fn || rank < 2 || rank > 3) return false;
   cuuint64_t d[3], st[2];
   cuuint32_t bx[3], es[3] = {1, 1, 1};
@@ -217,7 +222,6 @@ DecodeArgs decode_args(const v4moe_config* cfg, int32_t T, const void* x, const 
   d.w = *weights;
   d.out = static_cast<__nv_bfloat16*>(out);
   d.status = at<uint32_t>(ws, L.status);
-  d.scores = at<float>(ws, L.scores);
   d.ctl = at<uint32_t>(ws, L.d_ctl);
   d.dh = at<__half>(ws, L.d_dh);
   d.hs = at<__half>(ws, L.d_hs);

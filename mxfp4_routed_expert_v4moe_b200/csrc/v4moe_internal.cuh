@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -32,7 +33,10 @@ int32_t check_device();
 int device_sms();
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link to
-// libcuda): a tiled map of rank 2 or 3 with unit element strides, no
+// libcuda), looked up once; null when the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// A tiled map of rank 2 or 3 with unit element strides, no
 // interleave, L2 promotion of 256 bytes and no fill. dims / box list the
 // innermost dimension first; strides[i] is the byte stride of dimension i + 1.
 // False when the entry point is missing or the driver rejects the map.
@@ -61,7 +65,7 @@ DecodeBuffers dec_buffers(const v4moe_config& c, int64_t T);
 // Workspace carve-up for T tokens. All offsets are 256-byte aligned.
 struct WsLayout {
   size_t status = 0;        // uint32 status word + spare words (256 B)
-  size_t scores = 0;        // router: [ksplit, T, E] fp32 partial logits; decode: [T, E] scores
+  size_t scores = 0;        // router: [ksplit, T, E] fp32 partial logits
   size_t chunk_counts = 0;  // [nchunks, E] int32
   size_t chunk_base = 0;    // [nchunks, E] int32
   size_t h = 0;             // [T*k, I] bf16 routed intermediates (sorted order)
@@ -206,7 +210,6 @@ struct DecodeArgs {
   int32_t* offsets;
   int32_t* sorted_slot;
   int32_t* slot_pos;
-  float* scores;
   v4moe_weights w;
   __nv_bfloat16* out;
   uint32_t* status;
